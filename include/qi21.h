@@ -1,0 +1,265 @@
+/*
+ * qi21.h — C ABI of the B200 (sm_100a) cached Flow-Matching Euler step of a
+ * single-stream, Qwen-Image-2.1-style diffusion transformer with a prefix K/V
+ * cache.
+ *
+ * Sources (course pages on Qwen-Image-2.1; section names as on the pages):
+ *   [LAB]  "Bài Lab tổng hợp — Qwen-Image-2.1 Architecture": the 1:1 mapping
+ *          table and the NumPy lab qwen-image-21.py, blocks [1A] .. [6B].
+ *   [E2E]  "Lab tổng hợp Qwen-Image-2.1 — chạy toàn trình 1A → 6B bằng NumPy",
+ *          §1 Định nghĩa, §3 Giải pháp, §4 Profiling.
+ *   [6B]   "6B · Scale-Only Final AdaLN, Dự đoán vận tốc v_θ & Vòng lặp 8-Step Euler".
+ *   [3B]   "3B · Điều kiện nhân quả (t=0 vs t) & Bộ điều biến dùng chung".
+ *   [2A]   "2A · Mở rộng 4× Slot ảnh & Ghép chuỗi đồng nhất".
+ *
+ * Conventions for every entry point
+ *   - Device pointers are plain CUDA device addresses owned by the caller. The
+ *     library never allocates or frees device memory; scratch comes from the
+ *     caller's workspace (see qi21_workspace_bytes).
+ *   - Work is enqueued on the given cudaStream_t (passed as void*; NULL is the
+ *     legacy default stream). No call synchronises the host except
+ *     qi21_check_device_error.
+ *   - Matrices are row-major. Weights use the torch.nn.Linear order
+ *     [out][in]; per-layer weights are stacked on a leading layer axis.
+ *   - Every device pointer must be 16-byte aligned; otherwise QI21_ERR_INVALID_ARG.
+ *   - Host-detectable errors return before anything is enqueued. A device-side
+ *     bounded wait that expires sets an error word in the workspace, the
+ *     kernel returns, and qi21_check_device_error reports QI21_ERR_DEVICE_TIMEOUT.
+ *   - Every function is thread-compatible (no hidden global state besides the
+ *     optional per-kernel timing of qi21_profile_*).
+ */
+#ifndef QI21_H
+#define QI21_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t qi21_status;
+enum {
+    QI21_OK = 0,
+    QI21_ERR_INVALID_ARG = 1,      /* null / misaligned pointer, bad enum value */
+    QI21_ERR_SHAPE = 2,            /* inconsistent sizes (d != H*Dh, N == 0 ...) */
+    QI21_ERR_METADATA = 3,         /* target not last, empty segment, bad coords */
+    QI21_ERR_CACHE_STATE = 4,      /* cached step before extract, or cache shape mismatch */
+    QI21_ERR_UNSUPPORTED = 5,      /* shape the selected kernel family does not cover */
+    QI21_ERR_CUDA = 6,             /* a CUDA runtime / driver call failed */
+    QI21_ERR_DEVICE_TIMEOUT = 7,   /* a bounded device wait expired */
+    QI21_ERR_WORKSPACE_TOO_SMALL = 8
+};
+
+/* Storage dtype of weights, activations and the K/V cache. The residual
+ * stream, LayerNorm statistics, softmax and all accumulators are fp32 in
+ * both modes. F32 runs CUDA-core kernels (the parity mode); BF16 runs the
+ * tcgen05 tensor-core GEMMs and attention (the throughput mode). */
+enum { QI21_DTYPE_F32 = 0, QI21_DTYPE_BF16 = 1 };
+
+/* Model configuration.
+ *   d_model = n_heads * head_dim; mlp_hidden = SwiGLU width; latent_ch = C
+ *   (64 in production, [LAB] 1A); time_dim = width of the sin-cos timestep
+ *   embedding ([3B] §1).
+ *   use_shift = 0: modulation rows hold 4 chunks [scale1, gate1, scale2, gate2]
+ *   ([3B] §1-§2, scale-only AdaLN). use_shift = 1: 6 chunks
+ *   [shift1, scale1, gate1, shift2, scale2, gate2] as in the NumPy lab
+ *   ([LAB] 3B); the modulated LayerNorm then adds the shift.
+ *   ln_eps: LayerNorm epsilon; qk_eps: QK-RMSNorm epsilon (1e-6 in [LAB]). */
+typedef struct {
+    int32_t d_model, n_heads, head_dim, n_layers, mlp_hidden, latent_ch, time_dim;
+    int32_t dtype;
+    int32_t use_shift;
+    float ln_eps, qk_eps;
+} qi21_config;
+
+/* One segment of the packed sequence ([2A] §1-§2): TEXT with n_text tokens,
+ * or IMAGE with an h x w latent grid (patch size 1, row-major). Condition
+ * images take ids 0..K-1 in order; the LAST segment must be the target image. */
+enum { QI21_SEG_TEXT = 0, QI21_SEG_IMAGE = 1 };
+typedef struct {
+    int32_t kind;
+    int32_t n_text;
+    int32_t h, w;
+} qi21_segment;
+
+/* Device weights (dtype of the config unless stated), [out][in] order.
+ *   w_img_in [d][C]        img_in, latent -> token ([LAB] 1A, patch size 1)
+ *   w_out    [C][d]        proj_out -> v_theta ([6B] §1)
+ *   w_t1     [d][time_dim], w_t2 [d][d]   timestep MLP ([3B] §1; shape is a reading)
+ *   w_mod    [chunks*d][d] shared modulation Linear ([3B] §1)
+ *   w_fin    [d][d]        final AdaLN scale Linear ([6B] §3)
+ *   w_q, w_k, w_v, w_o     [L][d][d]
+ *   w_gate, w_up           [L][F][d]
+ *   w_down                 [L][d][F]
+ *   q_norm, k_norm         [L][head_dim] float32: QK-RMSNorm weights w, applied as (1 + w). */
+typedef struct {
+    const void *w_img_in, *w_out;
+    const void *w_t1, *w_t2, *w_mod, *w_fin;
+    const void *w_q, *w_k, *w_v, *w_o;
+    const void *w_gate, *w_up, *w_down;
+    const float *q_norm, *k_norm;
+} qi21_weights;
+
+/* Prefix K/V cache ([LAB] 6A; [E2E] §6 "kv_cache_mode"): one caller-owned
+ * device buffer of qi21_kv_cache_bytes(), laid out [L][2 (K,V)][B][P+N][d]
+ * in the config dtype. For layer l, item b, row r, head h, dim j the K value
+ * sits at ((l*2 + 0)*B + b)*(P+N)*d + r*d + h*head_dim + j. Rows [0, P) hold
+ * the prefix K (after QK-RMSNorm and RoPE) and raw V written by
+ * qi21_prefix_extract; rows [P, P+N) are rewritten by every cached step with
+ * that step's target K/V. state: QI21_CACHE_EMPTY until an extract succeeds. */
+enum { QI21_CACHE_EMPTY = 0, QI21_CACHE_EXTRACTED = 1 };
+typedef struct {
+    void *base;
+    int32_t batch, n_prefix, n_target;
+    int32_t n_layers, d_model, dtype;
+    int32_t state;
+} qi21_kv_cache;
+
+/* ---------------------------------------------------------------- host helpers */
+
+/* Packing metadata of a segment list ([2A] §1 build_token_metadata; [LAB] 3A,
+ * 3C). Host-only and pure. Outputs (each caller-allocated host array of S
+ * entries, any may be NULL): image_ids (-1 text, 0..K-1 condition images, K
+ * target), target_mask (1 on target tokens), coords [S][3] = (frame, h, w)
+ * (text (i,i,i) counting text tokens; images frame 0 — or the image id when
+ * frame_mode = 1 — and grid r - H/2, c - W/2), kv_limit (row q may attend to
+ * keys [0, kv_limit[q]): q+1 for text, the end of its image's run otherwise;
+ * exactly the block-causal rule (q >= kv) or same image id).
+ * Pass image_ids = NULL etc. with capacity 0 to query S, P, N first.
+ * Returns QI21_ERR_METADATA if the last segment is not an image, a segment is
+ * empty, or capacity < S. */
+qi21_status qi21_build_metadata(const qi21_segment *segments, int32_t n_segments,
+                                int32_t frame_mode, int32_t capacity,
+                                int32_t *image_ids, uint8_t *target_mask,
+                                int32_t *coords, int32_t *kv_limit,
+                                int32_t *S, int32_t *P, int32_t *N);
+
+/* Axial RoPE frequencies omega [head_dim/2][3] (host). Production split
+ * ([LAB] 3A notes): head_dim 128 -> (frame 16, height 56, width 56) dims,
+ * i.e. 8 + 28 + 28 pairs, omega = base^(-2j/dim_axis); other head dims scale
+ * the split by head_dim/128 (head_dim % 16 == 0). */
+qi21_status qi21_rope_omega_axial(int32_t head_dim, double base, double *omega);
+
+/* cos/sin table [S][head_dim/2][2] float32 (host, computed in fp64): angle of
+ * pair j at token s = sum_a coords[s][a] * omega[j][a]; entry = (cos, sin).
+ * The kernels rotate adjacent pairs (2j, 2j+1) as in [LAB] 3A. */
+qi21_status qi21_rope_table(int32_t head_dim, const int32_t *coords, int32_t S,
+                            const double *omega, float *cos_sin);
+
+/* Sin-cos timestep embedding [time_dim] (host, fp64 math, float result):
+ * [cos(t f_i) ..., sin(t f_i) ...], f_i = 10000^(-2i/time_dim), t = 1000*sigma
+ * ([LAB] 3B, [3B] §1). */
+qi21_status qi21_timestep_embedding(double t, int32_t time_dim, float *emb);
+
+/* Sizes in bytes of the caller-allocated buffers. */
+size_t qi21_kv_cache_bytes(const qi21_config *cfg, int32_t batch, int32_t n_prefix, int32_t n_target);
+/* Workspace large enough for every entry point with these sizes
+ * (the full recompute over S = P + N tokens is the largest). */
+size_t qi21_workspace_bytes(const qi21_config *cfg, int32_t batch, int32_t n_prefix, int32_t n_target);
+
+/* Initialise a cache descriptor over caller memory (state EMPTY). */
+qi21_status qi21_kv_cache_init(qi21_kv_cache *cache, void *base, const qi21_config *cfg,
+                               int32_t batch, int32_t n_prefix, int32_t n_target);
+
+/* ---------------------------------------------------------------- device entry points */
+
+/* Shared modulation ([3B] §1-§2; [6B] §3): for timestep t (= 1000*sigma),
+ *   e = w_t2 . silu(w_t1 . emb(t)),  mod_row = w_mod . silu(e)  [chunks*d],
+ *   scale_final = w_fin . silu(e)  [d]   (device float32 outputs).
+ * The prefix row is mod_row at t = 0 (computed once per image); the target
+ * row is recomputed every step. ws: workspace of >= qi21_workspace_bytes. */
+qi21_status qi21_modulation(const qi21_config *cfg, const qi21_weights *w, double t,
+                            float *mod_row, float *scale_final,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* Prefix extract ([LAB] 6A mode "extract"; [E2E] §3): run the L blocks over
+ * the P prefix rows of every batch item with the prefix modulation row (t = 0
+ * under causal_condition, [3B] §1) and the block-causal mask given as
+ * kv_limit_prefix [P] (device int32, from qi21_build_metadata), writing K
+ * (post QK-RMSNorm, post RoPE) and V of every layer into cache rows [0, P).
+ *   prefix_hidden  [B][P][d] float32 device (joint hidden states of the prefix)
+ *   cos_sin_prefix [P][head_dim/2][2] float32 device
+ *   mod_row_prefix [chunks*d] float32 device
+ * On success cache->state = QI21_CACHE_EXTRACTED. */
+qi21_status qi21_prefix_extract(const qi21_config *cfg, const qi21_weights *w,
+                                qi21_kv_cache *cache, const float *prefix_hidden,
+                                const float *cos_sin_prefix, const int32_t *kv_limit_prefix,
+                                const float *mod_row_prefix,
+                                void *ws, size_t ws_bytes, void *stream);
+
+/* Cached step ([LAB] 6A mode "cached", 6B; [E2E] §3): v_theta for the N
+ * target tokens of every item. Only target rows run the blocks: img_in(x_k),
+ * then per block LN(h)(1+scale1) -> Q,K,V -> QK-RMSNorm -> RoPE -> attention
+ * over [cached prefix K/V; this step's target K/V] (all P+N keys: the target
+ * is last) -> h += tanh(gate1)(o Wo) -> LN(h)(1+scale2) -> SwiGLU ->
+ * h += tanh(gate2)(. Wdown); then v = (LN(h)(1+scale_final)) Wout.
+ *   x_k            [B][N][C] float32 device (current latent, standardised space)
+ *   cos_sin_target [N][head_dim/2][2] float32 device
+ *   mod_row_target [chunks*d], scale_final [d] float32 device (from qi21_modulation)
+ *   v_out          [B][N][C] float32 device
+ * Returns QI21_ERR_CACHE_STATE unless the cache was extracted with matching
+ * sizes. Writes cache rows [P, P+N) (target K/V of this step). */
+qi21_status qi21_cached_step(const qi21_config *cfg, const qi21_weights *w,
+                             const qi21_kv_cache *cache, const float *x_k,
+                             const float *cos_sin_target, const float *mod_row_target,
+                             const float *scale_final, float *v_out,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* Full recomputation ([LAB] run_pipeline with use_cache=False; [E2E] §4):
+ * every one of the S = P + N tokens runs every block with the block-causal
+ * mask (kv_limit_all [S] device int32); prefix rows read mod_row_prefix,
+ * target rows mod_row_target ([3B] _select_modulation_rows). No cache is
+ * read or written (K/V live in the workspace). Used to check the cache path.
+ *   prefix_hidden [B][P][d] f32, x_k [B][N][C] f32, cos_sin_all [S][Dh/2][2] f32,
+ *   v_out [B][N][C] f32. */
+qi21_status qi21_full_recompute_step(const qi21_config *cfg, const qi21_weights *w,
+                                     int32_t batch, int32_t n_prefix, int32_t n_target,
+                                     const float *prefix_hidden, const float *x_k,
+                                     const float *cos_sin_all, const int32_t *kv_limit_all,
+                                     const float *mod_row_prefix, const float *mod_row_target,
+                                     const float *scale_final, float *v_out,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* Flow-Match Euler update ([6B] §1): x_out = x_k + (sigma_k1 - sigma_k) * v,
+ * n float32 elements; the difference is formed in fp64 on the host.
+ * x_out may alias x_k. */
+qi21_status qi21_euler_update(const float *x_k, const float *v, double sigma_k, double sigma_k1,
+                              float *x_out, int64_t n, void *stream);
+
+/* Synchronise the stream, then read and clear the device error word of the
+ * workspace. Returns QI21_OK, QI21_ERR_DEVICE_TIMEOUT or QI21_ERR_CUDA. */
+qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *stream);
+
+const char *qi21_status_string(qi21_status s);
+
+/* ---------------------------------------------------------------- per-kernel timing */
+
+/* When enabled, the entry points record a CUDA event pair on their stream
+ * around every kernel launch, grouped by kernel name. qi21_profile_read
+ * synchronises the recorded events and returns, for each kernel name, the
+ * launch count and total milliseconds (names are static strings).
+ * Returns the number of entries written. Off by default. */
+typedef struct {
+    const char *name;
+    int64_t launches;
+    double total_ms;
+} qi21_kernel_time;
+void qi21_profile_enable(int32_t enable);
+int32_t qi21_profile_read(qi21_kernel_time *out, int32_t max_entries);
+void qi21_profile_reset(void);
+
+/* Kernel family of the BF16 mode: 1 (default) the tcgen05 tensor-core GEMMs
+ * and attention; 0 the CUDA-core kernels of the F32 mode run on bf16 storage
+ * (differential testing of the two families). Process-wide. */
+void qi21_set_tensor_cores(int32_t enable);
+
+/* Library version string and the number of kernels the last entry point call
+ * enqueued (for launch accounting). */
+const char *qi21_version(void);
+int32_t qi21_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QI21_H */

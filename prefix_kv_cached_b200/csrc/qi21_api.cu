@@ -1,0 +1,543 @@
+// C-ABI entry points: argument validation, workspace carve-up and the per-layer
+// launch sequence of the prefix extract, the cached step and the full
+// recomputation (see include/qi21.h for the contract of each call).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "qi21.h"
+#include "qi21_internal.h"
+#include "qi21_simt.cuh"
+#include "qi21_tc.cuh"
+
+bool qi21_config_ok(const qi21_config *c);
+
+namespace qi21 {
+
+// ------------------------------------------------------------------ per-kernel timing
+struct ProfRec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static bool g_prof_on = false;
+static std::vector<cudaEvent_t> g_event_pool;
+static size_t g_event_next = 0;
+static std::vector<ProfRec> g_prof_recs;
+static int g_last_launches = 0;
+static bool g_tc_enabled = true;
+
+static cudaEvent_t prof_event() {
+    if (g_event_next == g_event_pool.size()) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+        g_event_pool.push_back(e);
+    }
+    return g_event_pool[g_event_next++];
+}
+
+struct Launcher {
+    cudaStream_t st;
+    int count = 0;
+    qi21_status status = QI21_OK;
+    explicit Launcher(cudaStream_t s) : st(s) {}
+    template <typename F>
+    void run(const char *name, F &&f) {
+        if (status != QI21_OK) return;
+        cudaEvent_t a = nullptr, b = nullptr;
+        if (g_prof_on) {
+            std::lock_guard<std::mutex> lk(g_prof_mu);
+            a = prof_event();
+            b = prof_event();
+        }
+        if (a) cudaEventRecord(a, st);
+        f();
+        ++count;
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) {
+            fprintf(stderr, "qi21: launch of %s failed: %s\n", name, cudaGetErrorString(e));
+            status = QI21_ERR_CUDA;
+            return;
+        }
+        if (b) {
+            cudaEventRecord(b, st);
+            std::lock_guard<std::mutex> lk(g_prof_mu);
+            g_prof_recs.push_back({name, a, b});
+        }
+    }
+    ~Launcher() { g_last_launches = count; }
+};
+
+static inline bool al16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
+
+static inline int grid_for(int64_t n, int threads, int cap = 148 * 16) {
+    int64_t g = (n + threads - 1) / threads;
+    if (g < 1) g = 1;
+    if (g > cap) g = cap;
+    return (int)g;
+}
+
+// ------------------------------------------------------------------ block stack
+struct StackArgs {
+    int B, M, split;          // items, rows per item in this call, rows < split read the prefix row
+    int P, N;                 // prefix / target sizes of the sequence
+    float *h;                 // fp32 [B*M][d]
+    void *xn, *q, *o, *hid;   // T buffers
+    float *gemm;              // fp32 scratch (F32 mode)
+    float *gates;             // [4][d]
+    uint32_t *err;
+    const float *mod_lo, *mod_hi;
+    const float *cos_sin;     // [M][Dh/2][2]
+    char *kv_k0, *kv_v0;      // K / V base of layer 0 (bytes)
+    int64_t kv_layer_stride;  // elements between layers (0: one buffer reused)
+    int64_t kv_bstride;       // elements between items
+    int row_off;              // K/V row of token 0 of this call
+    int kv_len;               // keys visible (rows of the K/V buffer per item)
+    const int *kv_limit;      // [M] or null
+    bool kv_only_last;        // extract: the last layer only needs K/V
+};
+
+template <typename T>
+static void launch_modln(Launcher &L, const qi21_config &c, const float *h, T *out, int rows, int M, int split,
+                         const float *sc_lo, const float *sc_hi, const float *sh_lo, const float *sh_hi) {
+    const int d = c.d_model;
+    if (d % 4 == 0 && d <= 4 * 256 * 8) {
+        const int vpt = (d / 4 + 255) / 256;
+        L.run("modln", [&] {
+#define QI21_LN(V)                                                                                           \
+    k_modln_vec<T, V><<<rows, 256, 0, L.st>>>(h, out, d, M, split, sc_lo, sc_hi, sh_lo, sh_hi, c.ln_eps)
+            if (vpt <= 1) QI21_LN(1);
+            else if (vpt <= 2) QI21_LN(2);
+            else if (vpt <= 4) QI21_LN(4);
+            else QI21_LN(8);
+#undef QI21_LN
+        });
+    } else {
+        L.run("modln", [&] {
+            k_modln_any<T><<<rows, 256, 0, L.st>>>(h, out, d, M, split, sc_lo, sc_hi, sh_lo, sh_hi, c.ln_eps);
+        });
+    }
+}
+
+template <typename T>
+static void launch_gemm_simt(Launcher &L, const T *A, int lda, const T *W, int ldw, float *Cm, int ldc, int M,
+                             int N, int K) {
+    dim3 grid((N + 63) / 64, (M + 63) / 64);
+    L.run("gemm_simt", [&] { k_gemm_simt<T><<<grid, 256, 0, L.st>>>(A, lda, W, ldw, Cm, ldc, M, N, K); });
+}
+
+template <typename T>
+static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, const StackArgs &a) {
+    const int d = c.d_model, F = c.mlp_hidden, H = c.n_heads, Dh = c.head_dim;
+    const int R = a.B * a.M;
+    const int ch_scale1 = c.use_shift ? 1 : 0, ch_scale2 = c.use_shift ? 4 : 2;
+    const float *sc1_lo = a.mod_lo + (size_t)ch_scale1 * d, *sc1_hi = a.mod_hi + (size_t)ch_scale1 * d;
+    const float *sc2_lo = a.mod_lo + (size_t)ch_scale2 * d, *sc2_hi = a.mod_hi + (size_t)ch_scale2 * d;
+    const float *sh1_lo = c.use_shift ? a.mod_lo : nullptr, *sh1_hi = c.use_shift ? a.mod_hi : nullptr;
+    const float *sh2_lo = c.use_shift ? a.mod_lo + 3 * (size_t)d : nullptr;
+    const float *sh2_hi = c.use_shift ? a.mod_hi + 3 * (size_t)d : nullptr;
+    const float *tg1_lo = a.gates, *tg1_hi = a.gates + d, *tg2_lo = a.gates + 2 * d, *tg2_hi = a.gates + 3 * d;
+    T *xn = (T *)a.xn, *q = (T *)a.q, *o = (T *)a.o, *hid = (T *)a.hid;
+    const bool tc = std::is_same<T, bf16>::value && g_tc_enabled && tc_supported(c);
+    const float scale = 1.0f / sqrtf((float)Dh);
+
+    L.run("prep_gates", [&] {
+        k_prep_gates<<<grid_for(d, 256), 256, 0, L.st>>>(a.mod_lo, a.mod_hi, d, c.use_shift, a.gates);
+    });
+    for (int l = 0; l < c.n_layers; ++l) {
+        const T *Wq = (const T *)w.w_q + (size_t)l * d * d, *Wk = (const T *)w.w_k + (size_t)l * d * d;
+        const T *Wv = (const T *)w.w_v + (size_t)l * d * d, *Wo = (const T *)w.w_o + (size_t)l * d * d;
+        const T *Wg = (const T *)w.w_gate + (size_t)l * F * d, *Wu = (const T *)w.w_up + (size_t)l * F * d;
+        const T *Wd = (const T *)w.w_down + (size_t)l * d * F;
+        const float *qn = w.q_norm + (size_t)l * Dh, *kn = w.k_norm + (size_t)l * Dh;
+        T *kdst = (T *)(a.kv_k0) + (size_t)l * a.kv_layer_stride;
+        T *vdst = (T *)(a.kv_v0) + (size_t)l * a.kv_layer_stride;
+
+        launch_modln<T>(L, c, a.h, xn, R, a.M, a.split, sc1_lo, sc1_hi, sh1_lo, sh1_hi);
+        if (tc) {
+            tc_gemm_qkv(L, c, (const bf16 *)xn, R, a.M, (const bf16 *)Wq, (const bf16 *)Wk, (const bf16 *)Wv, qn, kn,
+                        a.cos_sin, (bf16 *)q, (bf16 *)kdst, (bf16 *)vdst, a.kv_bstride, a.row_off, a.err);
+        } else {
+            launch_gemm_simt<T>(L, xn, d, Wq, d, a.gemm, 3 * d, R, d, d);
+            launch_gemm_simt<T>(L, xn, d, Wk, d, a.gemm + d, 3 * d, R, d, d);
+            launch_gemm_simt<T>(L, xn, d, Wv, d, a.gemm + 2 * d, 3 * d, R, d, d);
+            L.run("qkv_post", [&] {
+                k_qkv_post<T><<<(R * H + 3) / 4, 128, 0, L.st>>>(a.gemm, R, a.M, d, H, Dh, qn, kn, c.qk_eps,
+                                                               a.cos_sin, q, kdst, vdst, a.kv_bstride, a.row_off);
+            });
+        }
+        if (a.kv_only_last && l == c.n_layers - 1) break;
+
+        if (tc) {
+            tc_attention(L, c, (const bf16 *)q, (int64_t)a.M * d, a.M, (const bf16 *)kdst, (const bf16 *)vdst,
+                         a.kv_bstride, a.kv_len, a.kv_limit, (bf16 *)o, a.B, a.err);
+        } else {
+            const size_t smem = sizeof(float) * (3 * 32 * (Dh + 1) + 32 * 33);
+            static bool attr_set = false;
+            if (!attr_set) {
+                cudaFuncSetAttribute(k_attn_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+                attr_set = true;
+            }
+            dim3 grid((a.M + 31) / 32, H, a.B);
+            L.run("attn_simt", [&] {
+                k_attn_simt<T><<<grid, 128, smem, L.st>>>(q, (int64_t)a.M * d, a.M, d, kdst, vdst, a.kv_bstride, d,
+                                                         a.kv_len, a.kv_limit, o, Dh, scale);
+            });
+        }
+        if (tc) {
+            tc_gemm_residual(L, c, (const bf16 *)o, R, d, (const bf16 *)Wo, d, a.h, a.M, a.split, tg1_lo, tg1_hi,
+                             a.err, "gemm_o");
+        } else {
+            launch_gemm_simt<T>(L, o, d, Wo, d, a.gemm, d, R, d, d);
+            L.run("gated_residual", [&] {
+                k_gated_residual<<<grid_for((int64_t)R * d, 256), 256, 0, L.st>>>(a.h, a.gemm, d, R, d, a.M, a.split,
+                                                                                   tg1_lo, tg1_hi);
+            });
+        }
+        launch_modln<T>(L, c, a.h, xn, R, a.M, a.split, sc2_lo, sc2_hi, sh2_lo, sh2_hi);
+        if (tc) {
+            tc_gemm_swiglu(L, c, (const bf16 *)xn, R, (const bf16 *)Wg, (const bf16 *)Wu, (bf16 *)hid, a.err);
+            tc_gemm_residual(L, c, (const bf16 *)hid, R, F, (const bf16 *)Wd, d, a.h, a.M, a.split, tg2_lo, tg2_hi,
+                             a.err, "gemm_down");
+        } else {
+            launch_gemm_simt<T>(L, xn, d, Wg, d, a.gemm, 2 * F, R, F, d);
+            launch_gemm_simt<T>(L, xn, d, Wu, d, a.gemm + F, 2 * F, R, F, d);
+            L.run("swiglu", [&] {
+                k_swiglu<T><<<grid_for((int64_t)R * F, 256), 256, 0, L.st>>>(a.gemm, hid, R, F);
+            });
+            launch_gemm_simt<T>(L, hid, F, Wd, F, a.gemm, d, R, d, F);
+            L.run("gated_residual", [&] {
+                k_gated_residual<<<grid_for((int64_t)R * d, 256), 256, 0, L.st>>>(a.h, a.gemm, d, R, d, a.M, a.split,
+                                                                                   tg2_lo, tg2_hi);
+            });
+        }
+    }
+}
+
+template <typename T>
+static void launch_img_in(Launcher &L, const qi21_config &c, const float *x, const void *w_img_in, float *h, int B,
+                          int N, int M_out, int off) {
+    const int rows = B * N, C = c.latent_ch, d = c.d_model;
+    dim3 grid((rows + 15) / 16, (d + 255) / 256);
+    L.run("img_in", [&] {
+        k_img_in<T><<<grid, 256, sizeof(float) * 16 * C, L.st>>>(x, (const T *)w_img_in, h, rows, C, d, N, M_out, off);
+    });
+}
+
+template <typename T>
+static void launch_final(Launcher &L, const qi21_config &c, const float *h, int M, int off, int B, int N,
+                         const float *sf, const void *w_out, float *v) {
+    const int rows = B * N, d = c.d_model;
+    const size_t smem = sizeof(float) * 4 * d;
+    static bool attr_set[2] = {false, false};
+    if (smem > 48 * 1024 && !attr_set[sizeof(T) == 2]) {
+        cudaFuncSetAttribute(k_final<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        attr_set[sizeof(T) == 2] = true;
+    }
+    L.run("final", [&] {
+        k_final<T><<<(rows + 3) / 4, 256, smem, L.st>>>(h, M, off, N, d, sf, (const T *)w_out, c.latent_ch, c.ln_eps,
+                                                       v, rows);
+    });
+}
+
+// ------------------------------------------------------------------ validation helpers
+static qi21_status check_weights(const qi21_weights *w, bool need_time) {
+    if (!w) return QI21_ERR_INVALID_ARG;
+    const void *ps[] = {w->w_img_in, w->w_out, w->w_q, w->w_k, w->w_v, w->w_o, w->w_gate, w->w_up, w->w_down,
+                        w->q_norm, w->k_norm};
+    for (const void *p : ps)
+        if (!al16(p)) return QI21_ERR_INVALID_ARG;
+    if (need_time) {
+        const void *ts[] = {w->w_t1, w->w_t2, w->w_mod, w->w_fin};
+        for (const void *p : ts)
+            if (!al16(p)) return QI21_ERR_INVALID_ARG;
+    }
+    return QI21_OK;
+}
+
+static qi21_status check_shapes(const qi21_config *c) {
+    if (!c) return QI21_ERR_INVALID_ARG;
+    if (!qi21_config_ok(c)) return QI21_ERR_SHAPE;
+    // 16-byte row alignment of every activation row and cos/sin row
+    if (c->d_model % 8 || c->mlp_hidden % 8 || c->latent_ch % 4 || c->head_dim % 4) return QI21_ERR_UNSUPPORTED;
+    if (c->head_dim > 128 || c->time_dim > 512) return QI21_ERR_UNSUPPORTED;
+    if (c->dtype == QI21_DTYPE_BF16 && g_tc_enabled && !tc_supported(*c)) return QI21_ERR_UNSUPPORTED;
+    return QI21_OK;
+}
+
+static qi21_status finish(Launcher &L) { return L.status; }
+
+}  // namespace qi21
+
+using namespace qi21;
+
+// ------------------------------------------------------------------ entry points
+extern "C" qi21_status qi21_modulation(const qi21_config *c, const qi21_weights *w, double t, float *mod_row,
+                                       float *scale_final, void *ws, size_t ws_bytes, void *stream) {
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    if (!w || !al16(w->w_t1) || !al16(w->w_t2) || !al16(w->w_mod) || !al16(w->w_fin)) return QI21_ERR_INVALID_ARG;
+    if (!al16(mod_row) || !al16(scale_final) || !al16(ws)) return QI21_ERR_INVALID_ARG;
+    if (!std::isfinite(t)) return QI21_ERR_INVALID_ARG;
+    const WsLayout lay = ws_layout(*c, 1, 0, 1);
+    if (ws_bytes < lay.modtmp + align256(sizeof(float) * 2 * c->d_model)) return QI21_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    const int d = c->d_model, K0 = c->time_dim, nch = c->use_shift ? 6 : 4;
+    TembArg emb;
+    qi21_timestep_embedding(t, K0, emb.v);
+    float *a1 = (float *)((char *)ws + lay.modtmp), *e = a1 + d;
+    const size_t xs = sizeof(float) * d;
+    if (c->dtype == QI21_DTYPE_BF16) {
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(k_gemv2<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            attr = true;
+        }
+        L.run("temb_in", [&] { k_temb_in<bf16><<<(d + 7) / 8, 256, 0, st>>>((const bf16 *)w->w_t1, emb, K0, d, a1); });
+        L.run("gemv", [&] {
+            k_gemv2<bf16><<<(d + 7) / 8, 256, xs, st>>>((const bf16 *)w->w_t2, d, e, (const bf16 *)w->w_t2, 0, e, a1, d, 0);
+        });
+        L.run("gemv", [&] {
+            k_gemv2<bf16><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const bf16 *)w->w_mod, nch * d, mod_row,
+                                                                  (const bf16 *)w->w_fin, d, scale_final, e, d, 1);
+        });
+    } else {
+        static bool attr = false;
+        if (!attr) {
+            cudaFuncSetAttribute(k_gemv2<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            attr = true;
+        }
+        L.run("temb_in", [&] { k_temb_in<float><<<(d + 7) / 8, 256, 0, st>>>((const float *)w->w_t1, emb, K0, d, a1); });
+        L.run("gemv", [&] {
+            k_gemv2<float><<<(d + 7) / 8, 256, xs, st>>>((const float *)w->w_t2, d, e, (const float *)w->w_t2, 0, e, a1,
+                                                          d, 0);
+        });
+        L.run("gemv", [&] {
+            k_gemv2<float><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const float *)w->w_mod, nch * d, mod_row,
+                                                                   (const float *)w->w_fin, d, scale_final, e, d, 1);
+        });
+    }
+    return finish(L);
+}
+
+extern "C" qi21_status qi21_prefix_extract(const qi21_config *c, const qi21_weights *w, qi21_kv_cache *cache,
+                                           const float *prefix_hidden, const float *cos_sin_prefix,
+                                           const int32_t *kv_limit_prefix, const float *mod_row_prefix, void *ws,
+                                           size_t ws_bytes, void *stream) {
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    if ((s = check_weights(w, false))) return s;
+    if (!cache || !al16(cache->base)) return QI21_ERR_INVALID_ARG;
+    if (!al16(prefix_hidden) || !al16(cos_sin_prefix) || !al16(kv_limit_prefix) || !al16(mod_row_prefix) ||
+        !al16(ws))
+        return QI21_ERR_INVALID_ARG;
+    const int B = cache->batch, P = cache->n_prefix, N = cache->n_target;
+    if (cache->n_layers != c->n_layers || cache->d_model != c->d_model || cache->dtype != c->dtype || B <= 0 ||
+        P <= 0 || N <= 0)
+        return QI21_ERR_CACHE_STATE;
+    const WsLayout lay = ws_layout(*c, B, P, N);
+    if (ws_bytes < lay.total) return QI21_ERR_WORKSPACE_TOO_SMALL;
+    char *wsb = (char *)ws;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    const int d = c->d_model;
+    const size_t eb = dtype_bytes(c->dtype);
+    cache->state = QI21_CACHE_EMPTY;
+    StackArgs a{};
+    a.B = B; a.M = P; a.split = P; a.P = P; a.N = N;
+    a.h = (float *)(wsb + lay.h);
+    a.xn = wsb + lay.xn; a.q = wsb + lay.q; a.o = wsb + lay.o; a.hid = wsb + lay.hid;
+    a.gemm = (float *)(wsb + lay.gemm); a.gates = (float *)(wsb + lay.gates); a.err = (uint32_t *)(wsb + lay.err);
+    a.mod_lo = mod_row_prefix; a.mod_hi = mod_row_prefix;
+    a.cos_sin = cos_sin_prefix;
+    const int64_t rows = (int64_t)P + N;
+    a.kv_k0 = (char *)cache->base;
+    a.kv_v0 = (char *)cache->base + eb * (size_t)B * rows * d;
+    a.kv_layer_stride = 2 * (int64_t)B * rows * d;
+    a.kv_bstride = rows * d;
+    a.row_off = 0;
+    a.kv_len = P;
+    a.kv_limit = kv_limit_prefix;
+    a.kv_only_last = true;
+    L.run("copy_prefix", [&] {
+        const int64_t tot = (int64_t)B * P * d;
+        k_copy_rows<<<grid_for(tot, 256), 256, 0, st>>>(prefix_hidden, a.h, P, d, P, tot);
+    });
+    if (c->dtype == QI21_DTYPE_BF16) run_stack<bf16>(L, *c, *w, a);
+    else run_stack<float>(L, *c, *w, a);
+    s = finish(L);
+    if (s == QI21_OK) cache->state = QI21_CACHE_EXTRACTED;
+    return s;
+}
+
+extern "C" qi21_status qi21_cached_step(const qi21_config *c, const qi21_weights *w, const qi21_kv_cache *cache,
+                                        const float *x_k, const float *cos_sin_target, const float *mod_row_target,
+                                        const float *scale_final, float *v_out, void *ws, size_t ws_bytes,
+                                        void *stream) {
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    if ((s = check_weights(w, false))) return s;
+    if (!cache || !al16(cache->base)) return QI21_ERR_INVALID_ARG;
+    if (!al16(x_k) || !al16(cos_sin_target) || !al16(mod_row_target) || !al16(scale_final) || !al16(v_out) ||
+        !al16(ws))
+        return QI21_ERR_INVALID_ARG;
+    if (cache->state != QI21_CACHE_EXTRACTED || cache->n_layers != c->n_layers || cache->d_model != c->d_model ||
+        cache->dtype != c->dtype)
+        return QI21_ERR_CACHE_STATE;
+    const int B = cache->batch, P = cache->n_prefix, N = cache->n_target;
+    const WsLayout lay = ws_layout(*c, B, P, N);
+    if (ws_bytes < lay.total) return QI21_ERR_WORKSPACE_TOO_SMALL;
+    char *wsb = (char *)ws;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    const int d = c->d_model;
+    const size_t eb = dtype_bytes(c->dtype);
+    StackArgs a{};
+    a.B = B; a.M = N; a.split = 0; a.P = P; a.N = N;
+    a.h = (float *)(wsb + lay.h);
+    a.xn = wsb + lay.xn; a.q = wsb + lay.q; a.o = wsb + lay.o; a.hid = wsb + lay.hid;
+    a.gemm = (float *)(wsb + lay.gemm); a.gates = (float *)(wsb + lay.gates); a.err = (uint32_t *)(wsb + lay.err);
+    a.mod_lo = mod_row_target; a.mod_hi = mod_row_target;
+    a.cos_sin = cos_sin_target;
+    const int64_t rows = (int64_t)P + N;
+    a.kv_k0 = (char *)cache->base;
+    a.kv_v0 = (char *)cache->base + eb * (size_t)B * rows * d;
+    a.kv_layer_stride = 2 * (int64_t)B * rows * d;
+    a.kv_bstride = rows * d;
+    a.row_off = P;
+    a.kv_len = (int)rows;
+    a.kv_limit = nullptr;
+    a.kv_only_last = false;
+    if (c->dtype == QI21_DTYPE_BF16) {
+        launch_img_in<bf16>(L, *c, x_k, w->w_img_in, a.h, B, N, N, 0);
+        run_stack<bf16>(L, *c, *w, a);
+        launch_final<bf16>(L, *c, a.h, N, 0, B, N, scale_final, w->w_out, v_out);
+    } else {
+        launch_img_in<float>(L, *c, x_k, w->w_img_in, a.h, B, N, N, 0);
+        run_stack<float>(L, *c, *w, a);
+        launch_final<float>(L, *c, a.h, N, 0, B, N, scale_final, w->w_out, v_out);
+    }
+    return finish(L);
+}
+
+extern "C" qi21_status qi21_full_recompute_step(const qi21_config *c, const qi21_weights *w, int32_t B, int32_t P,
+                                                int32_t N, const float *prefix_hidden, const float *x_k,
+                                                const float *cos_sin_all, const int32_t *kv_limit_all,
+                                                const float *mod_row_prefix, const float *mod_row_target,
+                                                const float *scale_final, float *v_out, void *ws, size_t ws_bytes,
+                                                void *stream) {
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    if ((s = check_weights(w, false))) return s;
+    if (B <= 0 || P <= 0 || N <= 0) return QI21_ERR_SHAPE;
+    if (!al16(prefix_hidden) || !al16(x_k) || !al16(cos_sin_all) || !al16(kv_limit_all) || !al16(mod_row_prefix) ||
+        !al16(mod_row_target) || !al16(scale_final) || !al16(v_out) || !al16(ws))
+        return QI21_ERR_INVALID_ARG;
+    const WsLayout lay = ws_layout(*c, B, P, N);
+    if (ws_bytes < lay.total) return QI21_ERR_WORKSPACE_TOO_SMALL;
+    char *wsb = (char *)ws;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    const int d = c->d_model, S = P + N;
+    const size_t eb = dtype_bytes(c->dtype);
+    StackArgs a{};
+    a.B = B; a.M = S; a.split = P; a.P = P; a.N = N;
+    a.h = (float *)(wsb + lay.h);
+    a.xn = wsb + lay.xn; a.q = wsb + lay.q; a.o = wsb + lay.o; a.hid = wsb + lay.hid;
+    a.gemm = (float *)(wsb + lay.gemm); a.gates = (float *)(wsb + lay.gates); a.err = (uint32_t *)(wsb + lay.err);
+    a.mod_lo = mod_row_prefix; a.mod_hi = mod_row_target;
+    a.cos_sin = cos_sin_all;
+    a.kv_k0 = wsb + lay.kvf;
+    a.kv_v0 = wsb + lay.kvf + eb * (size_t)B * S * d;
+    a.kv_layer_stride = 0;
+    a.kv_bstride = (int64_t)S * d;
+    a.row_off = 0;
+    a.kv_len = S;
+    a.kv_limit = kv_limit_all;
+    a.kv_only_last = false;
+    L.run("copy_prefix", [&] {
+        const int64_t tot = (int64_t)B * P * d;
+        k_copy_rows<<<grid_for(tot, 256), 256, 0, st>>>(prefix_hidden, a.h, P, d, S, tot);
+    });
+    if (c->dtype == QI21_DTYPE_BF16) {
+        launch_img_in<bf16>(L, *c, x_k, w->w_img_in, a.h, B, N, S, P);
+        run_stack<bf16>(L, *c, *w, a);
+        launch_final<bf16>(L, *c, a.h, S, P, B, N, scale_final, w->w_out, v_out);
+    } else {
+        launch_img_in<float>(L, *c, x_k, w->w_img_in, a.h, B, N, S, P);
+        run_stack<float>(L, *c, *w, a);
+        launch_final<float>(L, *c, a.h, S, P, B, N, scale_final, w->w_out, v_out);
+    }
+    return finish(L);
+}
+
+extern "C" qi21_status qi21_euler_update(const float *x_k, const float *v, double sigma_k, double sigma_k1,
+                                         float *x_out, int64_t n, void *stream) {
+    if (!al16(x_k) || !al16(v) || !al16(x_out) || n < 0) return QI21_ERR_INVALID_ARG;
+    if (!std::isfinite(sigma_k) || !std::isfinite(sigma_k1)) return QI21_ERR_INVALID_ARG;
+    if (n == 0) return QI21_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    const float dsig = (float)(sigma_k1 - sigma_k);
+    L.run("euler", [&] { k_euler<<<grid_for((n + 3) / 4, 256), 256, 0, st>>>(x_k, v, dsig, x_out, n); });
+    return finish(L);
+}
+
+extern "C" qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *stream) {
+    if (!al16(ws) || ws_bytes < 64) return QI21_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return QI21_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return QI21_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return QI21_ERR_CUDA;
+        cudaStreamSynchronize(st);
+        return QI21_ERR_DEVICE_TIMEOUT;
+    }
+    return QI21_OK;
+}
+
+extern "C" void qi21_profile_enable(int32_t enable) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = enable != 0;
+}
+
+extern "C" void qi21_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_recs.clear();
+    g_event_next = 0;
+}
+
+extern "C" int32_t qi21_profile_read(qi21_kernel_time *out, int32_t max_entries) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    std::vector<qi21_kernel_time> acc;
+    for (const ProfRec &r : g_prof_recs) {
+        cudaEventSynchronize(r.b);
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, r.a, r.b);
+        bool found = false;
+        for (auto &k : acc)
+            if (strcmp(k.name, r.name) == 0) {
+                k.launches += 1;
+                k.total_ms += ms;
+                found = true;
+                break;
+            }
+        if (!found) acc.push_back({r.name, 1, (double)ms});
+    }
+    int32_t n = 0;
+    for (auto &k : acc) {
+        if (n >= max_entries || !out) break;
+        out[n++] = k;
+    }
+    return n;
+}
+
+extern "C" int32_t qi21_last_launch_count(void) { return g_last_launches; }
+
+extern "C" void qi21_set_tensor_cores(int32_t enable) { g_tc_enabled = enable != 0; }

@@ -1,0 +1,55 @@
+// Internal declarations shared by the host helpers and the CUDA entry points.
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include "qi21.h"
+
+namespace qi21 {
+
+// Workspace carve-up. Every region starts on a 256-byte boundary.
+//   err     : device error words (uint32 [8])
+//   gates   : fp32 [4][d]  tanh(gate1) prefix row, tanh(gate1) target row,
+//                          tanh(gate2) prefix row, tanh(gate2) target row
+//   modtmp  : fp32 [2][d]  timestep-MLP intermediates
+//   h       : fp32 [R][d]  residual stream (R = B * S rows at most)
+//   xn      : T [R][d]     modulated LayerNorm output (LN1 and LN2 share it)
+//   q       : T [R][d]     queries after QK-RMSNorm and RoPE
+//   o       : T [R][d]     attention output
+//   hid     : T [R][F]     SwiGLU activation
+//   kvf     : T [2][B][S][d]  K/V of the full recomputation
+//   gemm    : fp32 [R][max(3d, 2F)]  CUDA-core path GEMM outputs (F32 mode only)
+struct WsLayout {
+    size_t err, gates, modtmp, h, xn, q, o, hid, kvf, gemm, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline size_t dtype_bytes(int32_t dtype) { return dtype == QI21_DTYPE_BF16 ? 2 : 4; }
+
+inline WsLayout ws_layout(const qi21_config &c, int64_t B, int64_t P, int64_t N) {
+    const int64_t S = P + N, R = B * S, d = c.d_model, F = c.mlp_hidden;
+    const size_t eb = dtype_bytes(c.dtype);
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    L.err = take(64);
+    L.gates = take(sizeof(float) * 4 * d);
+    L.modtmp = take(sizeof(float) * 2 * d);
+    L.h = take(sizeof(float) * R * d);
+    L.xn = take(eb * R * d);
+    L.q = take(eb * R * d);
+    L.o = take(eb * R * d);
+    L.hid = take(eb * R * F);
+    L.kvf = take(eb * 2 * B * S * d);
+    const int64_t gw = (3 * d > 2 * F) ? 3 * d : 2 * F;
+    L.gemm = take(c.dtype == QI21_DTYPE_F32 ? sizeof(float) * R * gw : 0);
+    L.total = off;
+    return L;
+}
+
+}  // namespace qi21

@@ -1,0 +1,146 @@
+"""Device-side driver of one model instance over the C ABI.
+
+Owns the torch-allocated device buffers (weights, K/V cache, workspace,
+metadata tables) and calls the library's entry points; it computes nothing
+itself. Weights come either from host arrays (exact stored values) or are
+drawn directly on the device with the seeded generator (large models).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+from qi21_synth import configs as C
+from qi21_synth.gen import normal_torch
+
+_TORCH_DTYPE = {B.QI21_DTYPE_F32: torch.float32, B.QI21_DTYPE_BF16: torch.bfloat16}
+
+
+def make_config(shape: C.ModelShape, dtype: int) -> B.qi21_config:
+    return B.qi21_config(shape.d_model, shape.n_heads, shape.head_dim, shape.n_layers, shape.mlp_hidden,
+                         shape.latent_ch, shape.time_dim, dtype, shape.use_shift, shape.ln_eps, shape.qk_eps)
+
+
+def lab_rope_omega(base: float = 10000.0) -> np.ndarray:
+    """Micro RoPE split of the lab (head_dim 4): pair 0 on the frame axis at
+    rate 1; pair 1 shared by height (base^-1) and width (base^-1.5)."""
+    return np.array([[1.0, 0.0, 0.0], [0.0, base ** -1.0, base ** -1.5]], dtype=np.float64)
+
+
+class Qi21Runner:
+    def __init__(self, workload: C.Workload, dtype: int = B.QI21_DTYPE_F32, device: str = "cuda",
+                 host_weights: Optional[Dict[str, np.ndarray]] = None, frame_mode: int = 0):
+        self.w = workload
+        self.shape = workload.shape
+        self.dtype = dtype
+        self.tdtype = _TORCH_DTYPE[dtype]
+        self.device = torch.device(device)
+        self.cfg = make_config(self.shape, dtype)
+        sh = self.shape
+        self.meta = B.qi21_build_metadata(list(workload.segments), frame_mode)
+        self.S, self.P, self.N = self.meta["S"], self.meta["P"], self.meta["N"]
+        assert (self.P, self.N) == (workload.n_prefix, workload.n_target)
+        self.Bn = workload.batch
+        omega = lab_rope_omega() if sh.rope == "lab" else B.qi21_rope_omega_axial(sh.head_dim)
+        cs = B.qi21_rope_table(sh.head_dim, self.meta["coords"], omega)
+        self.cos_sin_all = torch.from_numpy(cs).to(self.device)
+        self.cos_sin_prefix = self.cos_sin_all[: self.P].contiguous()
+        self.cos_sin_target = self.cos_sin_all[self.P:].contiguous()
+        lim = torch.from_numpy(self.meta["kv_limit"].astype(np.int32)).to(self.device)
+        self.kv_limit_all = lim
+        self.kv_limit_prefix = lim[: self.P].contiguous()
+        self.weights: Dict[str, torch.Tensor] = {}
+        for name, shp in C.weight_specs(sh):
+            sdt = torch.float32 if name in ("q_norm", "k_norm") else self.tdtype
+            if host_weights is not None:
+                self.weights[name] = torch.from_numpy(np.ascontiguousarray(host_weights[name])).to(
+                    device=self.device, dtype=sdt)
+            else:
+                self.weights[name] = self._draw_weight(name, shp, sdt)
+        self.wstruct = B.qi21_weights(*[self.weights[n].data_ptr() for n in (
+            "w_img_in", "w_out", "w_t1", "w_t2", "w_mod", "w_fin", "w_q", "w_k", "w_v", "w_o", "w_gate", "w_up",
+            "w_down", "q_norm", "k_norm")])
+        kvb = B.qi21_kv_cache_bytes(self.cfg, self.Bn, self.P, self.N)
+        self.cache_buf = torch.zeros(kvb, dtype=torch.uint8, device=self.device)
+        self.cache = B.qi21_kv_cache_init(self.cache_buf, self.cfg, self.Bn, self.P, self.N)
+        self.ws_bytes = B.qi21_workspace_bytes(self.cfg, self.Bn, self.P, self.N)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        nch = sh.n_chunks
+        self.mod_prefix = torch.zeros(nch * sh.d_model, dtype=torch.float32, device=self.device)
+        self.mod_target = torch.zeros_like(self.mod_prefix)
+        self.scale_final = torch.zeros(sh.d_model, dtype=torch.float32, device=self.device)
+        self._sf0 = torch.zeros_like(self.scale_final)
+
+    def _draw_weight(self, name, shp, sdt):
+        w = self.w
+        if len(shp) == 3 or name in ("q_norm", "k_norm"):
+            out = torch.empty(shp, dtype=sdt, device=self.device)
+            for l in range(shp[0]):
+                out[l] = normal_torch(w.seed, f"L{l}.{name}", shp[1:], std=w.weight_std, device=self.device,
+                                      dtype=torch.float32).to(sdt)
+            return out
+        return normal_torch(w.seed, name, shp, std=w.weight_std, device=self.device,
+                            dtype=torch.float32).to(sdt)
+
+    @property
+    def stream(self) -> int:
+        return torch.cuda.current_stream(self.device).cuda_stream
+
+    # ------------------------------------------------------------------ calls
+    def modulation(self, t: float, mod_row: torch.Tensor, scale_final: torch.Tensor):
+        B.check("qi21_modulation", B.qi21_modulation(self.cfg, self.wstruct, t, mod_row, scale_final, self.ws,
+                                                     self.ws_bytes, self.stream))
+
+    def set_prefix_row(self):
+        """Prefix modulation row at t = 0 (3B page: prefix tokens read t = 0)."""
+        self.modulation(0.0, self.mod_prefix, self._sf0)
+
+    def set_target_row(self, sigma: float):
+        self.modulation(1000.0 * float(sigma), self.mod_target, self.scale_final)
+
+    def prefix_extract(self, prefix_hidden: torch.Tensor, mod_prefix: Optional[torch.Tensor] = None):
+        B.check("qi21_prefix_extract", B.qi21_prefix_extract(
+            self.cfg, self.wstruct, self.cache, prefix_hidden, self.cos_sin_prefix, self.kv_limit_prefix,
+            self.mod_prefix if mod_prefix is None else mod_prefix, self.ws, self.ws_bytes, self.stream))
+
+    def cached_step(self, x: torch.Tensor, v_out: torch.Tensor):
+        B.check("qi21_cached_step", B.qi21_cached_step(
+            self.cfg, self.wstruct, self.cache, x, self.cos_sin_target, self.mod_target, self.scale_final, v_out,
+            self.ws, self.ws_bytes, self.stream))
+
+    def full_recompute(self, prefix_hidden: torch.Tensor, x: torch.Tensor, v_out: torch.Tensor,
+                       mod_prefix: Optional[torch.Tensor] = None):
+        B.check("qi21_full_recompute_step", B.qi21_full_recompute_step(
+            self.cfg, self.wstruct, self.Bn, self.P, self.N, prefix_hidden, x, self.cos_sin_all, self.kv_limit_all,
+            self.mod_prefix if mod_prefix is None else mod_prefix, self.mod_target, self.scale_final, v_out,
+            self.ws, self.ws_bytes, self.stream))
+
+    def euler(self, x: torch.Tensor, v: torch.Tensor, s0: float, s1: float, x_out: torch.Tensor):
+        B.check("qi21_euler_update", B.qi21_euler_update(x, v, s0, s1, x_out, x.numel(), self.stream))
+
+    def check_device(self):
+        B.check("qi21_check_device_error", B.qi21_check_device_error(self.ws, self.ws_bytes, self.stream))
+
+    def cache_kv(self):
+        """Views of the cache as K, V [L][B][P+N][H][Dh] (for tests)."""
+        sh = self.shape
+        t = self.cache_buf.view(self.tdtype).view(sh.n_layers, 2, self.Bn, self.P + self.N, sh.n_heads,
+                                                  sh.head_dim)
+        return t[:, 0], t[:, 1]
+
+    def denoise(self, prefix_hidden: torch.Tensor, x0: torch.Tensor, sigmas=None):
+        """Whole image: t = 0 prefix row, extract once, then cached steps + Euler."""
+        sigmas = self.w.sigmas if sigmas is None else sigmas
+        self.set_prefix_row()
+        self.prefix_extract(prefix_hidden)
+        x = x0.clone()
+        v = torch.empty_like(x)
+        for k in range(len(sigmas) - 1):
+            self.set_target_row(sigmas[k])
+            self.cached_step(x, v)
+            self.euler(x, v, sigmas[k], sigmas[k + 1], x)
+        return x

@@ -1,0 +1,131 @@
+"""C-ABI library checks that need no GPU: it builds, loads, exports every
+symbol include/*.h declares, its host helpers agree with the oracle (bit-exact
+for integer metadata), and host-detectable errors return before any launch."""
+import ctypes as ct
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+from tests.conftest import ROOT
+from oracle import qi21_oracle as O
+from qi21_synth import configs as C
+
+
+@pytest.fixture(scope="module")
+def B():
+    from prefix_kv_cached_b200 import build
+    build.build()
+    from prefix_kv_cached_b200 import binding
+    return binding
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(qi21_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(B):
+    names = _declared_symbols()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(B.lib, n), f"{n} declared in include/ but not exported"
+    assert set(B.EXPORTED) <= set(names)
+
+
+@pytest.mark.parametrize("name", ["toy", "small", "small64", "full", "large"])
+def test_metadata_bit_exact_vs_oracle(B, name):
+    w = C.make_workload(name)
+    m = B.qi21_build_metadata(list(w.segments))
+    ids, mask, s, p, n = O.token_metadata(w.segments)
+    assert (m["S"], m["P"], m["N"]) == (s, p, n)
+    np.testing.assert_array_equal(m["image_ids"], ids)
+    np.testing.assert_array_equal(m["target_mask"].astype(bool), mask)
+    np.testing.assert_array_equal(m["coords"], O.rope_coords(w.segments))
+    if s <= 2000:
+        np.testing.assert_array_equal(m["kv_limit"], O.kv_limit_from_mask(O.block_causal_allowed(ids)))
+    m1 = B.qi21_build_metadata(list(w.segments), frame_mode=1)
+    np.testing.assert_array_equal(m1["coords"], O.rope_coords(w.segments, frame_mode=1))
+
+
+def test_toy_metadata_matches_page(B, golden):
+    g = golden("toy_sequence.json")
+    m = B.qi21_build_metadata([tuple(s) for s in g["segments"]])
+    assert m["image_ids"].tolist() == g["image_ids"]
+    assert m["kv_limit"].tolist() == g["mask_row_key_counts"]
+
+
+def test_rope_helpers_vs_oracle(B):
+    for dh in (64, 128):
+        np.testing.assert_array_equal(B.qi21_rope_omega_axial(dh), O.rope_omega_axial(dh))
+    w = C.make_workload("small")
+    m = B.qi21_build_metadata(list(w.segments))
+    om = O.rope_omega_axial(128)
+    cs = B.qi21_rope_table(128, m["coords"], om)
+    ang = O.rope_angles(m["coords"], om)
+    np.testing.assert_allclose(cs[..., 0], np.cos(ang), atol=6e-8)
+    np.testing.assert_allclose(cs[..., 1], np.sin(ang), atol=6e-8)
+    emb = B.qi21_timestep_embedding(850.0, 256)
+    np.testing.assert_allclose(emb, O.timestep_embedding(850.0, 256), atol=6e-8)
+
+
+def test_metadata_errors(B):
+    segs = (B.qi21_segment * 2)(B.qi21_segment(B.QI21_SEG_IMAGE, 0, 2, 2), B.qi21_segment(B.QI21_SEG_TEXT, 3, 0, 0))
+    S, P, N = ct.c_int32(), ct.c_int32(), ct.c_int32()
+    st = B.lib.qi21_build_metadata(segs, 2, 0, 0, None, None, None, None, ct.byref(S), ct.byref(P), ct.byref(N))
+    assert st == B.QI21_ERR_METADATA          # target must be last
+    segs2 = (B.qi21_segment * 1)(B.qi21_segment(B.QI21_SEG_IMAGE, 0, 0, 3))
+    assert B.lib.qi21_build_metadata(segs2, 1, 0, 0, None, None, None, None, ct.byref(S), ct.byref(P),
+                                     ct.byref(N)) == B.QI21_ERR_METADATA
+    ids = np.zeros(2, np.int32)
+    segs3 = (B.qi21_segment * 1)(B.qi21_segment(B.QI21_SEG_IMAGE, 0, 2, 2))
+    assert B.lib.qi21_build_metadata(segs3, 1, 0, 2, ids.ctypes.data, None, None, None, ct.byref(S), ct.byref(P),
+                                     ct.byref(N)) == B.QI21_ERR_METADATA    # capacity < S
+
+
+def _cfg(B, dtype=0):
+    from prefix_kv_cached_b200.runner import make_config
+    return make_config(C.SMALL, dtype)
+
+
+def test_host_validation_returns_before_launch(B):
+    cfg = _cfg(B)
+    fake = 0x10000          # aligned, never dereferenced on these paths
+    w = B.qi21_weights(*([fake] * 15))
+    cache = B.qi21_kv_cache_init(fake, cfg, 1, 8, 4)
+    ws_bytes = B.qi21_workspace_bytes(cfg, 1, 8, 4)
+    assert ws_bytes > 0 and B.qi21_kv_cache_bytes(cfg, 1, 8, 4) == 4 * 2 * 2 * 12 * 256
+    # cached step before any extract
+    assert B.qi21_cached_step(cfg, w, cache, fake, fake, fake, fake, fake, fake, ws_bytes, 0) == \
+        B.QI21_ERR_CACHE_STATE
+    # misaligned input pointer
+    cache.state = B.QI21_CACHE_EXTRACTED
+    assert B.qi21_cached_step(cfg, w, cache, fake + 4, fake, fake, fake, fake, fake, ws_bytes, 0) == \
+        B.QI21_ERR_INVALID_ARG
+    # workspace too small
+    assert B.qi21_cached_step(cfg, w, cache, fake, fake, fake, fake, fake, fake, ws_bytes - 1, 0) == \
+        B.QI21_ERR_WORKSPACE_TOO_SMALL
+    # cache built for another model
+    other = _cfg(B)
+    other.n_layers = 3
+    assert B.qi21_cached_step(other, w, cache, fake, fake, fake, fake, fake, fake, ws_bytes, 0) == \
+        B.QI21_ERR_CACHE_STATE
+    # inconsistent config
+    bad = _cfg(B)
+    bad.n_heads = 3
+    assert B.qi21_cached_step(bad, w, cache, fake, fake, fake, fake, fake, fake, ws_bytes, 0) == B.QI21_ERR_SHAPE
+    # null weight pointer
+    w2 = B.qi21_weights(*([fake] * 14 + [0]))
+    assert B.qi21_prefix_extract(cfg, w2, cache, fake, fake, fake, fake, fake, ws_bytes, 0) == \
+        B.QI21_ERR_INVALID_ARG
+    assert B.qi21_full_recompute_step(cfg, w, 0, 8, 4, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                                      ws_bytes, 0) == B.QI21_ERR_SHAPE
+    assert B.qi21_euler_update(fake, fake, 1.0, float("nan"), fake, 4, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_status_string(B.QI21_ERR_DEVICE_TIMEOUT).startswith("device wait")
