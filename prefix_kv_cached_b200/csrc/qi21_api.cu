@@ -1,6 +1,8 @@
 // C-ABI entry points: argument validation, workspace carve-up and the per-layer
 // launch sequence of the prefix extract, the cached step and the full
 // recomputation (see include/qi21.h for the contract of each call).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -12,7 +14,7 @@
 #include "qi21.h"
 #include "qi21_internal.h"
 #include "qi21_simt.cuh"
-#include "qi21_tc.cuh"
+#include "qi21_gemm_tc.cuh"
 
 bool qi21_config_ok(const qi21_config *c);
 
@@ -81,6 +83,86 @@ static inline int grid_for(int64_t n, int threads, int cap = 148 * 16) {
     return (int)g;
 }
 
+
+// ------------------------------------------------------------------ tensor-core family (BF16 mode)
+static bool tc_supported(const qi21_config &c) {
+    return c.dtype == QI21_DTYPE_BF16 && c.d_model % TC_BN == 0 && c.mlp_hidden % 128 == 0 &&
+           (c.head_dim == 64 || c.head_dim == 128) && c.d_model >= TC_BN;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+static bool get_encode() {
+    if (g_encode) return true;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+    g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    return true;
+}
+
+// 3-D bf16 tensor map over [depth][rows][inner] with a box of 64 x box_rows x 1,
+// 128-byte swizzle, zero fill outside the tensor.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t depth,
+                     uint32_t box_rows) {
+    if (!get_encode()) return false;
+    cuuint64_t dims[3] = {inner, rows, depth};
+    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int EPI>
+static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, const CUtensorMap &b0,
+                           const CUtensorMap &b1, const CUtensorMap &b2, const GemmParams &p) {
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(k_gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM_BYTES);
+        attr = true;
+    }
+    const int tiles = p.m_blocks * p.n_blocks;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, TC_SMEM_BYTES, L.st>>>(a, b0, b1, b2, p); });
+}
+
+struct TcMaps {
+    CUtensorMap xn, o, hid, wq, wk, wv, wo, wg, wu, wd;
+};
+
+static bool build_tc_maps(TcMaps &t, const qi21_config &c, const qi21_weights &w, const void *xn, const void *o,
+                          const void *hid, int R) {
+    const uint64_t d = c.d_model, F = c.mlp_hidden, L = c.n_layers;
+    bool ok = true;
+    ok &= make_map(&t.xn, xn, d, R, 1, 128);
+    ok &= make_map(&t.o, o, d, R, 1, 128);
+    ok &= make_map(&t.hid, hid, F, R, 1, 128);
+    ok &= make_map(&t.wq, w.w_q, d, d, L, 128);
+    ok &= make_map(&t.wk, w.w_k, d, d, L, 128);
+    ok &= make_map(&t.wv, w.w_v, d, d, L, 128);
+    ok &= make_map(&t.wo, w.w_o, d, d, L, 128);
+    ok &= make_map(&t.wg, w.w_gate, d, F, L, 128);
+    ok &= make_map(&t.wu, w.w_up, d, F, L, 128);
+    ok &= make_map(&t.wd, w.w_down, F, d, L, 128);
+    return ok;
+}
+
 // ------------------------------------------------------------------ block stack
 struct StackArgs {
     int B, M, split;          // items, rows per item in this call, rows < split read the prefix row
@@ -145,6 +227,31 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
     const bool tc = std::is_same<T, bf16>::value && g_tc_enabled && tc_supported(c);
     const float scale = 1.0f / sqrtf((float)Dh);
 
+    TcMaps maps;
+    GemmParams gp{};
+    if (tc) {
+        if (!build_tc_maps(maps, c, w, a.xn, a.o, a.hid, R)) {
+            L.status = QI21_ERR_CUDA;
+            return;
+        }
+        gp.R = R;
+        gp.m_blocks = (R + TC_BM - 1) / TC_BM;
+        gp.M = a.M;
+        gp.split = a.split;
+        gp.h = a.h;
+        gp.ldh = d;
+        gp.F = F;
+        gp.hid = (bf16 *)a.hid;
+        gp.d = d;
+        gp.Dh = Dh;
+        gp.qk_eps = c.qk_eps;
+        gp.cos_sin = a.cos_sin;
+        gp.q_out = (bf16 *)a.q;
+        gp.kv_bstride = a.kv_bstride;
+        gp.row_off = a.row_off;
+        gp.err = a.err;
+    }
+
     L.run("prep_gates", [&] {
         k_prep_gates<<<grid_for(d, 256), 256, 0, L.st>>>(a.mod_lo, a.mod_hi, d, c.use_shift, a.gates);
     });
@@ -156,11 +263,18 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         const float *qn = w.q_norm + (size_t)l * Dh, *kn = w.k_norm + (size_t)l * Dh;
         T *kdst = (T *)(a.kv_k0) + (size_t)l * a.kv_layer_stride;
         T *vdst = (T *)(a.kv_v0) + (size_t)l * a.kv_layer_stride;
+        gp.layer = l;
 
         launch_modln<T>(L, c, a.h, xn, R, a.M, a.split, sc1_lo, sc1_hi, sh1_lo, sh1_hi);
         if (tc) {
-            tc_gemm_qkv(L, c, (const bf16 *)xn, R, a.M, (const bf16 *)Wq, (const bf16 *)Wk, (const bf16 *)Wv, qn, kn,
-                        a.cos_sin, (bf16 *)q, (bf16 *)kdst, (bf16 *)vdst, a.kv_bstride, a.row_off, a.err);
+            GemmParams g = gp;
+            g.K = d;
+            g.n_blocks = 3 * d / TC_BN;
+            g.qn = qn;
+            g.kn = kn;
+            g.k_base = (bf16 *)kdst;
+            g.v_base = (bf16 *)vdst;
+            launch_gemm_tc<EPI_QKV>(L, "gemm_qkv", maps.xn, maps.wq, maps.wk, maps.wv, g);
         } else {
             launch_gemm_simt<T>(L, xn, d, Wq, d, a.gemm, 3 * d, R, d, d);
             launch_gemm_simt<T>(L, xn, d, Wk, d, a.gemm + d, 3 * d, R, d, d);
@@ -172,10 +286,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         }
         if (a.kv_only_last && l == c.n_layers - 1) break;
 
-        if (tc) {
-            tc_attention(L, c, (const bf16 *)q, (int64_t)a.M * d, a.M, (const bf16 *)kdst, (const bf16 *)vdst,
-                         a.kv_bstride, a.kv_len, a.kv_limit, (bf16 *)o, a.B, a.err);
-        } else {
+        {
             const size_t smem = sizeof(float) * (3 * 32 * (Dh + 1) + 32 * 33);
             static bool attr_set = false;
             if (!attr_set) {
@@ -189,8 +300,12 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             });
         }
         if (tc) {
-            tc_gemm_residual(L, c, (const bf16 *)o, R, d, (const bf16 *)Wo, d, a.h, a.M, a.split, tg1_lo, tg1_hi,
-                             a.err, "gemm_o");
+            GemmParams g = gp;
+            g.K = d;
+            g.n_blocks = d / TC_BN;
+            g.g_lo = tg1_lo;
+            g.g_hi = tg1_hi;
+            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.wo, g);
         } else {
             launch_gemm_simt<T>(L, o, d, Wo, d, a.gemm, d, R, d, d);
             L.run("gated_residual", [&] {
@@ -200,9 +315,16 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         }
         launch_modln<T>(L, c, a.h, xn, R, a.M, a.split, sc2_lo, sc2_hi, sh2_lo, sh2_hi);
         if (tc) {
-            tc_gemm_swiglu(L, c, (const bf16 *)xn, R, (const bf16 *)Wg, (const bf16 *)Wu, (bf16 *)hid, a.err);
-            tc_gemm_residual(L, c, (const bf16 *)hid, R, F, (const bf16 *)Wd, d, a.h, a.M, a.split, tg2_lo, tg2_hi,
-                             a.err, "gemm_down");
+            GemmParams g = gp;
+            g.K = d;
+            g.n_blocks = F / 128;
+            launch_gemm_tc<EPI_SWIGLU>(L, "gemm_gateup", maps.xn, maps.wg, maps.wu, maps.wu, g);
+            GemmParams g2 = gp;
+            g2.K = F;
+            g2.n_blocks = d / TC_BN;
+            g2.g_lo = tg2_lo;
+            g2.g_hi = tg2_hi;
+            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.wd, g2);
         } else {
             launch_gemm_simt<T>(L, xn, d, Wg, d, a.gemm, 2 * F, R, F, d);
             launch_gemm_simt<T>(L, xn, d, Wu, d, a.gemm + F, 2 * F, R, F, d);

@@ -1,0 +1,324 @@
+// Persistent warp-specialised tcgen05 GEMM with fused epilogues (BF16 mode).
+//
+//   D[r][n] = sum_k A[r][k] * W[n][k]      A: activations [R][K] bf16 (K-major)
+//                                          W: weights [N][K] bf16 (K-major, [out][in])
+// Tile 128 x 256 x 64, 4-stage TMA -> shared memory pipeline, fp32
+// accumulators double-buffered in TMEM (2 x 256 columns), one CTA per SM.
+//   warp 0      : TMA producer (one elected lane)
+//   warp 1      : TMEM allocator + UMMA issuer (one lane)
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31, i.e. one
+//                 output row per thread, 32 columns per tcgen05.ld.
+// Epilogues (the lab's [4A]/[5A] block):
+//   EPI_QKV      per-head zero-centred RMSNorm (1 + w) of q and k, RoPE on the
+//                adjacent pairs, q -> q buffer, k / v -> K/V rows of the cache
+//   EPI_RESIDUAL h[r][n] += tanh(gate)[n] * D[r][n]   (fp32 residual stream)
+//   EPI_SWIGLU   hid[r][j] = silu(D[r][j]) * D[r][F + j]   (gate and up halves
+//                of one 256-column tile come from W_gate and W_up rows j0..j0+127)
+#pragma once
+#include "qi21_sm100.cuh"
+
+namespace qi21 {
+
+enum { EPI_QKV = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2 };
+
+constexpr int TC_BM = 128, TC_BN = 256, TC_BK = 64, TC_STAGES = 4;
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;          // 16 KB
+constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;          // 32 KB
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
+constexpr int TC_THREADS = 192;
+constexpr size_t TC_SMEM_BYTES = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + 256;
+
+struct GemmParams {
+    int R;             // rows of A (tokens of all items)
+    int K;             // reduction length
+    int m_blocks;      // ceil(R / 128)
+    int n_blocks;      // output tiles along N
+    int M, split;      // rows per item; rows m < split read the prefix modulation row
+    // EPI_RESIDUAL
+    float *h;
+    int ldh;
+    const float *g_lo, *g_hi;
+    // EPI_SWIGLU
+    bf16 *hid;
+    int F;
+    // EPI_QKV
+    int d, Dh;
+    const float *qn, *kn;
+    float qk_eps;
+    const float *cos_sin;
+    bf16 *q_out, *k_base, *v_base;
+    int64_t kv_bstride;
+    int row_off;
+    int layer;         // z coordinate of the stacked weight tensor maps
+    uint32_t *err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// Store 32 fp32 values as bf16 (64 contiguous bytes, 16-byte aligned).
+__device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 u;
+        u.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+        u.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+        u.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+        u.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+        d4[i] = u;
+    }
+}
+
+template <int EPI>
+__device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int &m_blk, int &n_blk) {
+    // m fastest: CTAs running together share a weight tile, activations stay in L2
+    m_blk = tile % p.m_blocks;
+    n_blk = tile / p.m_blocks;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+              const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2, GemmParams p) {
+    using namespace sm100;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *stage_base = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)TC_STAGES * TC_STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + TC_STAGES, *tfull = bars + 2 * TC_STAGES, *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.m_blocks * p.n_blocks;
+    const int kblocks = p.K / TC_BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 128);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        tma_prefetch_desc(&tmB1);
+        if (EPI == EPI_QKV) tma_prefetch_desc(&tmB2);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                int m_blk, n_blk;
+                tile_coords<EPI>(p, tile, m_blk, n_blk);
+                const CUtensorMap *b0 = &tmB0, *b1 = &tmB1;
+                int rb0, rb1;
+                if (EPI == EPI_SWIGLU) {
+                    rb0 = rb1 = n_blk * 128;
+                } else if (EPI == EPI_QKV) {
+                    const int n0 = n_blk * TC_BN, part = n0 / p.d;
+                    const CUtensorMap *bm = part == 0 ? &tmB0 : (part == 1 ? &tmB1 : &tmB2);
+                    b0 = b1 = bm;
+                    rb0 = n0 - part * p.d;
+                    rb1 = rb0 + 128;
+                } else {
+                    rb0 = n_blk * TC_BN;
+                    rb1 = rb0 + 128;
+                }
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, TC_STAGE_BYTES);
+                    const uint32_t sa = smem_u32(stage_base + (size_t)stage * TC_STAGE_BYTES);
+                    const uint32_t sb = sa + TC_A_BYTES;
+                    tma_load_3d(sa, &tmA, fb, kb * TC_BK, m_blk * TC_BM, 0);
+                    tma_load_3d(sb, b0, fb, kb * TC_BK, rb0, p.layer);
+                    tma_load_3d(sb + TC_B_BYTES / 2, b1, fb, kb * TC_BK, rb1, p.layer);
+                    if (++stage == TC_STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- UMMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(stage_base + (size_t)stage * TC_STAGE_BYTES);
+                    const uint32_t sb = sa + TC_A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < TC_BK / 16; ++k) {
+                        umma_f16(d_tmem, sdesc_kmajor_sw128(sa + k * 32), sdesc_kmajor_sw128(sb + k * 32), idesc,
+                                 (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == TC_STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (ok) umma_commit(smem_u32(&tfull[acc]));
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue (warps 2..5)
+        const int quad = warp & 3;
+        const int row_in_tile = quad * 32 + lane;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+            int m_blk, n_blk;
+            tile_coords<EPI>(p, tile, m_blk, n_blk);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.err)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * TC_BN);
+            const int r = m_blk * TC_BM + row_in_tile;
+            const bool live = r < p.R;
+            const int m = live ? r % p.M : 0;
+            const int b = live ? r / p.M : 0;
+            float v[32];
+            if (EPI == EPI_RESIDUAL) {
+                const int n0 = n_blk * TC_BN;
+                const float *g = (m < p.split ? p.g_lo : p.g_hi) + n0;
+                float *hp = p.h + (size_t)r * p.ldh + n0;
+#pragma unroll 1
+                for (int cc = 0; cc < TC_BN / 32; ++cc) {
+                    tmem_ld32(t_row + cc * 32, v);
+                    tmem_wait_ld();
+                    if (live) {
+                        float4 *h4 = reinterpret_cast<float4 *>(hp + cc * 32);
+                        const float4 *g4 = reinterpret_cast<const float4 *>(g + cc * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float4 hv = h4[i];
+                            const float4 gv = g4[i];
+                            hv.x = fmaf(gv.x, v[4 * i + 0], hv.x);
+                            hv.y = fmaf(gv.y, v[4 * i + 1], hv.y);
+                            hv.z = fmaf(gv.z, v[4 * i + 2], hv.z);
+                            hv.w = fmaf(gv.w, v[4 * i + 3], hv.w);
+                            h4[i] = hv;
+                        }
+                    }
+                }
+            } else if (EPI == EPI_SWIGLU) {
+                const int j0 = n_blk * 128;
+                float u[32];
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    tmem_ld32(t_row + cc * 32, v);
+                    tmem_ld32(t_row + 128 + cc * 32, u);
+                    tmem_wait_ld();
+                    if (live) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i])) * u[i];
+                        store_bf16x32(p.hid + (size_t)r * p.F + j0 + cc * 32, v);
+                    }
+                }
+            } else {  // EPI_QKV
+                const int n0 = n_blk * TC_BN, part = n0 / p.d, c0 = n0 - part * p.d;
+                const int nch = p.Dh / 32;
+                if (part == 2) {
+                    bf16 *dst = p.v_base + (size_t)b * p.kv_bstride + (size_t)(p.row_off + m) * p.d + c0;
+#pragma unroll 1
+                    for (int cc = 0; cc < TC_BN / 32; ++cc) {
+                        tmem_ld32(t_row + cc * 32, v);
+                        tmem_wait_ld();
+                        if (live) store_bf16x32(dst + cc * 32, v);
+                    }
+                } else {
+                    const float *wn = part == 0 ? p.qn : p.kn;
+                    bf16 *dst_row = part == 0 ? p.q_out + (size_t)r * p.d
+                                              : p.k_base + (size_t)b * p.kv_bstride + (size_t)(p.row_off + m) * p.d;
+                    const float *cs_row = p.cos_sin + (size_t)m * p.Dh;   // [Dh/2][2] floats = Dh floats
+#pragma unroll 1
+                    for (int hh = 0; hh < TC_BN / p.Dh; ++hh) {
+                        float ss = 0.f;
+#pragma unroll 1
+                        for (int cc = 0; cc < nch; ++cc) {
+                            tmem_ld32(t_row + hh * p.Dh + cc * 32, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+                        }
+                        const float inv = rsqrtf(ss / (float)p.Dh + p.qk_eps);
+#pragma unroll 1
+                        for (int cc = 0; cc < nch; ++cc) {
+                            tmem_ld32(t_row + hh * p.Dh + cc * 32, v);
+                            tmem_wait_ld();
+                            if (live) {
+                                const float4 *w4 = reinterpret_cast<const float4 *>(wn + cc * 32);
+                                const float4 *cs4 = reinterpret_cast<const float4 *>(cs_row + cc * 32);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    const float4 w = w4[i];
+                                    const float4 cs = cs4[i];   // (cos, sin) of two pairs
+                                    const float y0 = v[4 * i + 0] * inv * (1.f + w.x);
+                                    const float y1 = v[4 * i + 1] * inv * (1.f + w.y);
+                                    const float y2 = v[4 * i + 2] * inv * (1.f + w.z);
+                                    const float y3 = v[4 * i + 3] * inv * (1.f + w.w);
+                                    v[4 * i + 0] = y0 * cs.x - y1 * cs.y;
+                                    v[4 * i + 1] = y0 * cs.y + y1 * cs.x;
+                                    v[4 * i + 2] = y2 * cs.z - y3 * cs.w;
+                                    v[4 * i + 3] = y2 * cs.w + y3 * cs.z;
+                                }
+                                store_bf16x32(dst_row + c0 + hh * p.Dh + cc * 32, v);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+}  // namespace qi21
