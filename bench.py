@@ -1,0 +1,447 @@
+"""Benchmark of the cached Flow-Matching Euler step (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the target-row
+modulation at this step's sigma, the cached step over the N target tokens of
+every item (all L blocks + final AdaLN + proj_out) and the Euler update. The
+prefix K/V cache is extracted once before timing (its cost is reported
+separately as part of the per-image figure). Inputs are seeded synthetic
+draws; the 14 GB of weights and the 4.6 GB K/V cache stream through HBM every
+step, so the working set is far larger than the 126 MB L2.
+
+With N > 1 (torchrun) every rank runs an independent replica (own weights,
+cache and latents); there is no collective in the data path, so scaling is
+weak and the value is the total over ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cached-step target tokens/s (d4096,L32); attn+GEMM % of bf16 tensor peak"
+UNIT = "target tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=16)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--workload", default="full")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def step_flops(w):
+    """Algorithmic FLOPs of one cached step (target tokens only):
+    per token per block 2*(4 d^2 + 3 d F) + 4 (P + N) d, plus img_in and proj_out."""
+    sh = w.shape
+    d, F, L, C = sh.d_model, sh.mlp_hidden, sh.n_layers, sh.latent_ch
+    ntok = w.batch * w.n_target
+    per_tok_block = 2 * (4 * d * d + 3 * d * F) + 4 * (w.n_prefix + w.n_target) * d
+    return ntok * (L * per_tok_block + 2 * 2 * d * C)
+
+
+def kernel_flops(w):
+    """Algorithmic FLOPs per launch of each tensor-core kernel of the cached step."""
+    sh = w.shape
+    d, F = sh.d_model, sh.mlp_hidden
+    R = w.batch * w.n_target
+    kv = w.n_prefix + w.n_target
+    return {
+        "gemm_qkv": 2 * R * d * 3 * d,
+        "gemm_o": 2 * R * d * d,
+        "gemm_gateup": 2 * R * d * 2 * F,
+        "gemm_down": 2 * R * F * d,
+        "attn": 4 * R * kv * d,
+        "attn_simt": 4 * R * kv * d,
+    }
+
+
+def kernel_bytes(w):
+    """Algorithmic HBM bytes per launch of the memory-bound kernels."""
+    sh = w.shape
+    d, C = sh.d_model, sh.latent_ch
+    R = w.batch * w.n_target
+    return {
+        "modln": R * d * (4 + 2),            # read fp32 h, write bf16
+        "img_in": R * C * 4 + R * d * 4,     # read x, write fp32 h
+        "final": R * d * 4 + R * C * 4,      # read h, write v
+        "euler": R * C * 12,
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "prefix_kv_cached_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for row in csv.reader(io.StringIO(out)):
+            if len(row) < 9:
+                continue
+            try:
+                sms.append(float(row[1]))
+                maxes.append(float(row[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, row[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sms) if sms else None,
+                "sm_max_mhz": max(maxes) if maxes else None,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+def oracle_sample(w, rows=512, seed=4321):
+    """Time the fp64 oracle on a bounded sample of the workload: one block of
+    the cached step at full width for `rows` target tokens attending to all
+    P + N keys (the other targets' K/V are synthetic cache rows). Returns
+    (seconds, target tokens/s scaled to all L blocks, threads, description)."""
+    from oracle import qi21_oracle as O
+
+    rows = min(rows, w.n_target)
+    sh = w.shape
+    d, F, H, Dh = sh.d_model, sh.mlp_hidden, sh.n_heads, sh.head_dim
+    rng = np.random.default_rng(seed)   # timing sample only: values are not compared with anything
+
+    def draw(name, shape, std):
+        return rng.standard_normal(shape) * std
+
+    lw = {"w_q": draw("wq", (d, d), 0.02), "w_k": draw("wk", (d, d), 0.02), "w_v": draw("wv", (d, d), 0.02),
+          "w_o": draw("wo", (d, d), 0.02), "w_gate": draw("wg", (F, d), 0.02), "w_up": draw("wu", (F, d), 0.02),
+          "w_down": draw("wd", (d, F), 0.02), "q_norm": draw("qn", (Dh,), 0.02), "k_norm": draw("kn", (Dh,), 0.02)}
+    extra = w.n_prefix + w.n_target - rows
+    kc = draw("kc", (extra, H, Dh), 1.0)
+    vc = draw("vc", (extra, H, Dh), 1.0)
+    h = draw("h", (rows, d), 1.0)
+    mods = O.split_chunks(draw("mod", (4 * d,), 0.1), 4)
+    coords = O.rope_coords(w.segments)[w.n_prefix:w.n_prefix + rows]
+    omega = O.rope_omega_axial(Dh)
+    allowed = np.ones((rows, extra + rows), dtype=bool)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    O.dit_block(h, mods, lw, H, coords, omega, (kc, vc), allowed, sh.ln_eps, sh.qk_eps)
+    dt = time.perf_counter() - t0
+    tok_s = rows / (dt * sh.n_layers)
+    desc = (f"one of {sh.n_layers} blocks of the cached step at d={d}, {rows} target rows attending to "
+            f"{w.n_prefix + w.n_target} keys, fp64 numpy; time x {sh.n_layers} blocks per token")
+    return dt, tok_s, threads, desc
+
+
+# ----------------------------------------------------------------------------- distributed helpers
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return 0
+    steps = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        dt, tok_s, threads, desc = oracle_sample(w)
+        if i >= args.warmup:
+            steps.append(dt)
+    dt = statistics.mean(steps)
+    rows = min(512, w.n_target)
+    tok_s = rows / (dt * w.shape.n_layers)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 * w.shape.n_layers * w.n_target / rows,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w),
+        "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    sh = w.shape
+    return {"workload": f"{w.name}: cached Flow-Matching Euler step, d={sh.d_model}, {sh.n_layers} blocks, "
+                        f"{sh.n_heads}x{sh.head_dim} heads, SwiGLU {sh.mlp_hidden}, {sh.latent_ch}-ch latents, "
+                        f"prefix {w.n_prefix} + target {w.n_target} tokens, batch {w.batch}",
+            "batch": w.batch, "n_prefix": w.n_prefix, "n_target": w.n_target, "sigmas": "Turbo 8-step",
+            "l2": "inputs larger than L2: every step streams 14 GB of weights and the K/V cache"}
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    args = parse()
+    from qi21_synth import configs as C
+    w = C.make_workload(args.workload)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = run_reference(args, w, world, rank)
+        dist_done(world)
+        return rc
+
+    import torch
+    from prefix_kv_cached_b200 import build as _build
+    if rank == 0:
+        _build.build()
+    dist_barrier(world)
+    from prefix_kv_cached_b200 import binding as B
+    from prefix_kv_cached_b200.runner import Qi21Runner
+    from qi21_synth.gen import normal_torch
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    seed_w = C.Workload(w.name, w.shape, w.batch, w.segments, w.sigmas, w.seed + 1000 * rank)
+    r = Qi21Runner(seed_w, B.QI21_DTYPE_BF16, device=str(dev))
+    sh = w.shape
+    pre = normal_torch(seed_w.seed, "prefix_hidden", (w.batch, w.n_prefix, sh.d_model), device=dev,
+                       dtype=torch.float32)
+    x0 = normal_torch(seed_w.seed, "noise", (w.batch, w.n_target, sh.latent_ch), device=dev, dtype=torch.float32)
+    x = x0.clone()
+    v = torch.empty_like(x)
+    sig = w.sigmas
+    st = torch.cuda.current_stream(dev)
+
+    # prefix extract (once per image), timed on its own
+    r.set_prefix_row()
+    r.prefix_extract(pre)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    r.prefix_extract(pre)
+    e1.record(st)
+    torch.cuda.synchronize()
+    extract_ms = e0.elapsed_time(e1)
+
+    launches = [0]
+
+    def step(k):
+        i = k % (len(sig) - 1)
+        r.set_target_row(sig[i])
+        n = B.qi21_last_launch_count()
+        r.cached_step(x, v)
+        n += B.qi21_last_launch_count()
+        r.euler(x, v, sig[i], sig[i + 1], x)
+        n += B.qi21_last_launch_count()
+        launches[0] += n
+
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    r.check_device()
+
+    clocks = ClockSampler(local)
+    B.qi21_profile_reset()
+    B.qi21_profile_enable(1)
+    launches[0] = 0
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(st)
+    for k in range(args.steps):
+        step(k)
+    t1.record(st)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    clk = clocks.stop()
+    B.qi21_profile_enable(0)
+    prof = B.qi21_profile_read()
+    ms = t0.elapsed_time(t1)
+    ms_max = dist_max(ms, world)
+    r.check_device()
+    ms_step = ms_max / args.steps
+    tokens = w.batch * w.n_target
+    value = world * tokens * args.steps / (ms_max / 1e3)
+
+    # e2e: same step through the C ABI with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.empty_like(x, device="cpu").pin_memory()
+        xh.copy_(x0.cpu())
+        xo = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(x)
+        for k in range(2):
+            xd.copy_(xh, non_blocking=True)
+            i = k % (len(sig) - 1)
+            r.set_target_row(sig[i]); r.cached_step(xd, v); r.euler(xd, v, sig[i], sig[i + 1], xd)
+            xo.copy_(xd, non_blocking=True)
+        torch.cuda.synchronize()
+        dist_barrier(world)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(st)
+        for k in range(args.steps):
+            xd.copy_(xh, non_blocking=True)
+            i = k % (len(sig) - 1)
+            r.set_target_row(sig[i]); r.cached_step(xd, v); r.euler(xd, v, sig[i], sig[i + 1], xd)
+            xo.copy_(xd, non_blocking=True)
+        a1.record(st)
+        torch.cuda.synchronize()
+        e_ms = dist_max(a0.elapsed_time(a1), world)
+        nbytes = x.numel() * 4
+        e2e = {"value": world * tokens * args.steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e_ms / args.steps}
+
+    if rank == 0:
+        peaks = load_peaks()
+        kf = kernel_flops(w)
+        kb = kernel_bytes(w)
+        kernels = {}
+        for name, (n, tot) in prof.items():
+            avg = tot / n
+            ent = {"launches": n, "total_ms": round(tot, 3), "avg_ms": round(avg, 4),
+                   "share": round(tot / sum(t for _, t in prof.values()), 4)}
+            if name in kf:
+                ach = kf[name] / (avg / 1e3) / 1e12
+                ent.update({"tflops": round(ach, 1), "frac_sustained": round(ach / peaks["bf16_tflops_sustained"], 3)})
+            elif name in kb:
+                ach = kb[name] / (avg / 1e3) / 1e9
+                ent.update({"gbs": round(ach, 1), "frac_hbm": round(ach / peaks["hbm_gbs"], 3)})
+            kernels[name] = ent
+        dom = max(((k, e) for k, e in kernels.items() if k in kf), key=lambda t: t[1]["total_ms"], default=None)
+        roof = None
+        if dom:
+            name, ent = dom
+            ach = kf[name] / (ent["avg_ms"] / 1e3) / 1e12
+            roof = {"kernel": name, "bound": "tensor", "achieved": round(ach, 1),
+                    "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "traffic": load_traffic(name),
+                    "peak_src": f"{peaks['src']} bf16 sustained (kernel timed inside a long step)",
+                    "algorithmic_flops_per_launch": kf[name]}
+        sflops = step_flops(w)
+        step_tflops = sflops / (ms_step / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64/Box-Muller draws)",
+            "config": config_dict(w),
+            "tensor_frac_step": round(step_tflops / peaks["bf16_tflops_sustained"], 4),
+            "step_tflops": round(step_tflops, 1),
+            "per_image": {"extract_ms": round(extract_ms, 3),
+                          "tokens_per_s": round(world * tokens / ((extract_ms + 8 * ms_step) / 1e3), 1)},
+            "roofline": roof, "kernels": kernels, "gpu_launches": launches[0], "clocks": clk, "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            dt, tok_s, threads, desc = oracle_sample(w)
+            line["cpu_baseline"] = {"value": round(tok_s, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": desc, "seconds": round(dt, 2)}
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
