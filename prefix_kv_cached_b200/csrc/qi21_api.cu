@@ -31,7 +31,6 @@ static std::vector<cudaEvent_t> g_event_pool;
 static size_t g_event_next = 0;
 static std::vector<ProfRec> g_prof_recs;
 static int g_last_launches = 0;
-static bool g_tc_enabled = true;
 
 static cudaEvent_t prof_event() {
     if (g_event_next == g_event_pool.size()) {
@@ -224,7 +223,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
     const float *sh2_hi = c.use_shift ? a.mod_hi + 3 * (size_t)d : nullptr;
     const float *tg1_lo = a.gates, *tg1_hi = a.gates + d, *tg2_lo = a.gates + 2 * d, *tg2_hi = a.gates + 3 * d;
     T *xn = (T *)a.xn, *q = (T *)a.q, *o = (T *)a.o, *hid = (T *)a.hid;
-    const bool tc = std::is_same<T, bf16>::value && g_tc_enabled && tc_supported(c);
+    const bool tc = std::is_same<T, bf16>::value && tc_enabled() && tc_supported(c);
     const float scale = 1.0f / sqrtf((float)Dh);
 
     TcMaps maps;
@@ -387,7 +386,7 @@ static qi21_status check_shapes(const qi21_config *c) {
     // 16-byte row alignment of every activation row and cos/sin row
     if (c->d_model % 8 || c->mlp_hidden % 8 || c->latent_ch % 4 || c->head_dim % 4) return QI21_ERR_UNSUPPORTED;
     if (c->head_dim > 128 || c->time_dim > 512) return QI21_ERR_UNSUPPORTED;
-    if (c->dtype == QI21_DTYPE_BF16 && g_tc_enabled && !tc_supported(*c)) return QI21_ERR_UNSUPPORTED;
+    if (c->dtype == QI21_DTYPE_BF16 && tc_enabled() && !tc_supported(*c)) return QI21_ERR_UNSUPPORTED;
     return QI21_OK;
 }
 
@@ -661,5 +660,3 @@ extern "C" int32_t qi21_profile_read(qi21_kernel_time *out, int32_t max_entries)
 }
 
 extern "C" int32_t qi21_last_launch_count(void) { return g_last_launches; }
-
-extern "C" void qi21_set_tensor_cores(int32_t enable) { g_tc_enabled = enable != 0; }

@@ -123,6 +123,10 @@ extern "C" const char *qi21_status_string(qi21_status s) {
 
 extern "C" const char *qi21_version(void) { return "qi21 0.1 sm_100a"; }
 
+static bool g_tc_enabled = true;
+bool qi21::tc_enabled() { return g_tc_enabled; }
+extern "C" void qi21_set_tensor_cores(int32_t enable) { g_tc_enabled = enable != 0; }
+
 bool qi21_config_ok(const qi21_config *c) {
     return c && c->d_model > 0 && c->n_heads > 0 && c->head_dim > 0 && c->n_layers > 0 &&
            c->mlp_hidden > 0 && c->latent_ch > 0 && c->time_dim > 0 && c->time_dim % 2 == 0 &&

@@ -18,7 +18,8 @@ namespace qi21 {
 //   o       : T [R][d]     attention output
 //   hid     : T [R][F]     SwiGLU activation
 //   kvf     : T [2][B][S][d]  K/V of the full recomputation
-//   gemm    : fp32 [R][max(3d, 2F)]  CUDA-core path GEMM outputs (F32 mode only)
+//   gemm    : fp32 [R][max(3d, 2F)]  outputs of the CUDA-core GEMMs (present when
+//             they run: F32 mode, or BF16 mode with the tensor cores switched off)
 struct WsLayout {
     size_t err, gates, modtmp, h, xn, q, o, hid, kvf, gemm, total;
 };
@@ -26,6 +27,11 @@ struct WsLayout {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 inline size_t dtype_bytes(int32_t dtype) { return dtype == QI21_DTYPE_BF16 ? 2 : 4; }
+
+// Kernel family of the BF16 mode (process-wide; qi21_set_tensor_cores).
+bool tc_enabled();
+
+inline bool uses_cuda_core_gemm(const qi21_config &c) { return c.dtype == QI21_DTYPE_F32 || !tc_enabled(); }
 
 inline WsLayout ws_layout(const qi21_config &c, int64_t B, int64_t P, int64_t N) {
     const int64_t S = P + N, R = B * S, d = c.d_model, F = c.mlp_hidden;
@@ -47,7 +53,7 @@ inline WsLayout ws_layout(const qi21_config &c, int64_t B, int64_t P, int64_t N)
     L.hid = take(eb * R * F);
     L.kvf = take(eb * 2 * B * S * d);
     const int64_t gw = (3 * d > 2 * F) ? 3 * d : 2 * F;
-    L.gemm = take(c.dtype == QI21_DTYPE_F32 ? sizeof(float) * R * gw : 0);
+    L.gemm = take(uses_cuda_core_gemm(c) ? sizeof(float) * R * gw : 0);
     L.total = off;
     return L;
 }

@@ -129,3 +129,25 @@ def test_host_validation_returns_before_launch(B):
                                       ws_bytes, 0) == B.QI21_ERR_SHAPE
     assert B.qi21_euler_update(fake, fake, 1.0, float("nan"), fake, 4, 0) == B.QI21_ERR_INVALID_ARG
     assert B.qi21_status_string(B.QI21_ERR_DEVICE_TIMEOUT).startswith("device wait")
+
+
+def test_workspace_covers_the_selected_kernel_family(B):
+    """BF16 with the tensor cores switched off runs the CUDA-core GEMMs, whose
+    fp32 outputs need extra workspace; a workspace sized for the tensor-core
+    family must then be refused before any launch."""
+    from prefix_kv_cached_b200.runner import make_config
+    cfg = make_config(C.SMALL, B.QI21_DTYPE_BF16)
+    tc_bytes = B.qi21_workspace_bytes(cfg, 2, 198, 300)
+    B.qi21_set_tensor_cores(0)
+    try:
+        cc_bytes = B.qi21_workspace_bytes(cfg, 2, 198, 300)
+        assert cc_bytes >= tc_bytes + 4 * 2 * 498 * 768
+        fake = 0x10000
+        w = B.qi21_weights(*([fake] * 15))
+        cache = B.qi21_kv_cache_init(fake, cfg, 2, 198, 300)
+        cache.state = B.QI21_CACHE_EXTRACTED
+        assert B.qi21_cached_step(cfg, w, cache, fake, fake, fake, fake, fake, fake, tc_bytes, 0) == \
+            B.QI21_ERR_WORKSPACE_TOO_SMALL
+    finally:
+        B.qi21_set_tensor_cores(1)
+    assert B.qi21_workspace_bytes(cfg, 2, 198, 300) == tc_bytes
