@@ -173,6 +173,27 @@ qi21_status qi21_modulation(const qi21_config *cfg, const qi21_weights *w, doubl
                             float *mod_row, float *scale_final,
                             void *ws, size_t ws_bytes, void *stream);
 
+/* Largest d_model qi21_modulation_noalloc accepts: its scratch is a fixed
+ * device array of 2 * QI21_NOALLOC_MAX_D floats (64 KB on every GPU that
+ * loads the library, held until the process exits). */
+#define QI21_NOALLOC_MAX_D 8192
+
+/* The pages have no counterpart to this call; it exists for callers of the
+ * library that cannot allocate device memory (their device memory is owned by
+ * another allocator, or they must never call cudaMalloc because it can block).
+ * Same result as qi21_modulation, but takes no workspace: its two
+ * timestep-MLP intermediate vectors live in a fixed file-scope device array of
+ * 2 * QI21_NOALLOC_MAX_D floats instead. Returns QI21_ERR_UNSUPPORTED when
+ * d_model > QI21_NOALLOC_MAX_D (or time_dim > 512), before anything is
+ * enqueued. Allocates nothing and calls no allocating routine. The first call
+ * on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current), so make that first call
+ * before any stream capture. Every call on a device shares the one array and
+ * overwrites what the previous call left there: calls that overlap on the GPU
+ * (for instance on two streams) race and must be serialised by the caller. */
+qi21_status qi21_modulation_noalloc(const qi21_config *cfg, const qi21_weights *w, double t,
+                                    float *mod_row, float *scale_final, void *stream);
+
 /* Prefix extract ([LAB] 6A mode "extract"; [E2E] §3): run the L blocks over
  * the P prefix rows of every batch item with the prefix modulation row (t = 0
  * under causal_condition, [3B] §1) and the block-causal mask given as

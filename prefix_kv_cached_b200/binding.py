@@ -71,6 +71,8 @@ _SIGS = {
     "qi21_kv_cache_init": (_I32, [ct.POINTER(qi21_kv_cache), _P, ct.POINTER(qi21_config), _I32, _I32, _I32]),
     "qi21_modulation": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P, _P,
                                ct.c_size_t, _P]),
+    "qi21_modulation_noalloc": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P,
+                                       _P]),
     "qi21_prefix_extract": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.POINTER(qi21_kv_cache),
                                    _P, _P, _P, _P, _P, ct.c_size_t, _P]),
     "qi21_cached_step": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.POINTER(qi21_kv_cache),
@@ -187,6 +189,11 @@ def qi21_kv_cache_init(base, cfg, batch, n_prefix, n_target):
 def qi21_modulation(cfg, weights, t, mod_row, scale_final, ws, ws_bytes, stream=0):
     return lib.qi21_modulation(ct.byref(cfg), ct.byref(weights), float(t), _addr(mod_row), _addr(scale_final),
                                _addr(ws), ws_bytes, stream)
+
+
+def qi21_modulation_noalloc(cfg, weights, t, mod_row, scale_final, stream=0):
+    return lib.qi21_modulation_noalloc(ct.byref(cfg), ct.byref(weights), float(t), _addr(mod_row),
+                                       _addr(scale_final), stream)
 
 
 def qi21_prefix_extract(cfg, weights, cache, prefix_hidden, cos_sin_prefix, kv_limit_prefix, mod_row_prefix,

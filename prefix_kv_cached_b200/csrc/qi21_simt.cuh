@@ -13,7 +13,7 @@ namespace qi21 {
 // [shift1, scale1, gate1, shift2, scale2, gate2] (lab [3B]).
 // gates = [tanh g1 prefix | tanh g1 target | tanh g2 prefix | tanh g2 target].
 // ---------------------------------------------------------------------------
-__global__ void k_prep_gates(const float *__restrict__ mod_lo, const float *__restrict__ mod_hi, int d,
+static __global__ void k_prep_gates(const float *__restrict__ mod_lo, const float *__restrict__ mod_hi, int d,
                              int use_shift, float *__restrict__ gates) {
     const int g1 = use_shift ? 2 : 1, g2 = use_shift ? 5 : 3;
     for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < d; c += gridDim.x * blockDim.x) {
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(256) k_img_in(const float *__restrict__ x, con
 }
 
 // Copy the prefix hidden states [B][P][d] into residual rows b*M_out + n.
-__global__ void k_copy_rows(const float *__restrict__ src, float *__restrict__ dst, int rows_per_item, int d,
+static __global__ void k_copy_rows(const float *__restrict__ src, float *__restrict__ dst, int rows_per_item, int d,
                             int M_out, int64_t total) {
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(128) k_qkv_post(const float *__restrict__ Cm, 
 }
 
 // h[r][c] += g[c] * Y[r][c], g = tanh(gate) of the row's modulation (lo/hi).
-__global__ void k_gated_residual(float *__restrict__ h, const float *__restrict__ Y, int ldy, int R, int d, int M,
+static __global__ void k_gated_residual(float *__restrict__ h, const float *__restrict__ Y, int ldy, int R, int d, int M,
                                  int split, const float *__restrict__ g_lo, const float *__restrict__ g_hi) {
     const int64_t total = (int64_t)R * d;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(256) k_final(const float *__restrict__ h, int 
 }
 
 // x_out = x + dsig * v  (6B page §1).
-__global__ void k_euler(const float *__restrict__ x, const float *__restrict__ v, float dsig,
+static __global__ void k_euler(const float *__restrict__ x, const float *__restrict__ v, float dsig,
                         float *__restrict__ xo, int64_t n) {
     const int64_t n4 = n >> 2;
     const float4 *x4 = reinterpret_cast<const float4 *>(x);
