@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqi21.so")
 SOURCES = ["qi21_api.cu", "qi21_noalloc.cu", "qi21_host.cpp"]
-HEADERS = ["qi21_internal.h", "qi21_common.cuh", "qi21_simt.cuh", "qi21_sm100.cuh", "qi21_gemm_tc.cuh"]
+HEADERS = ["qi21_internal.h", "qi21_common.cuh", "qi21_simt.cuh", "qi21_sm100.cuh", "qi21_gemm_tc.cuh", "qi21_attn_tc.cuh"]
 
 
 def _nvcc() -> str:

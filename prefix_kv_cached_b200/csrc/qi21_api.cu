@@ -15,6 +15,7 @@
 #include "qi21_internal.h"
 #include "qi21_simt.cuh"
 #include "qi21_gemm_tc.cuh"
+#include "qi21_attn_tc.cuh"
 
 bool qi21_config_ok(const qi21_config *c);
 
@@ -141,8 +142,35 @@ static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, 
     L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, TC_SMEM_BYTES, L.st>>>(a, b0, b1, b2, p); });
 }
 
+// 4-D bf16 tensor map [w][z][rows][inner] (strides in elements), box 64 x 128 x 1 x 1.
+static bool make_map4(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t zn, uint64_t wn,
+                      uint64_t row_stride, uint64_t z_stride, uint64_t w_stride) {
+    if (!get_encode()) return false;
+    cuuint64_t dims[4] = {inner, rows, zn, wn};
+    cuuint64_t strides[3] = {row_stride * 2, z_stride * 2, w_stride * 2};
+    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int DH>
+static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                           const AttnParams &p, int B) {
+    using Cf = AttnCfg<DH>;
+    static bool attr = false;
+    if (!attr) {
+        cudaFuncSetAttribute(k_attn_tc<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
+        attr = true;
+    }
+    dim3 grid((p.Mq + Cf::BQ - 1) / Cf::BQ, p.H, B);
+    L.run("attn", [&] { k_attn_tc<DH><<<grid, Cf::THREADS, Cf::SMEM, L.st>>>(q, k, v, p); });
+}
+
 struct TcMaps {
-    CUtensorMap xn, o, hid, wq, wk, wv, wo, wg, wu, wd;
+    CUtensorMap xn, o, hid, wq, wk, wv, wo, wg, wu, wd, q4, k4, v4;
 };
 
 static bool build_tc_maps(TcMaps &t, const qi21_config &c, const qi21_weights &w, const void *xn, const void *o,
@@ -233,6 +261,16 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             L.status = QI21_ERR_CUDA;
             return;
         }
+        // attention operands: q [R][d]; K and V [layer][item][kv_len rows][d]
+        const uint64_t nl = a.kv_layer_stride ? (uint64_t)c.n_layers : 1;
+        const uint64_t lstride = a.kv_layer_stride ? (uint64_t)a.kv_layer_stride : (uint64_t)a.kv_bstride * a.B;
+        bool ok = make_map4(&maps.q4, a.q, d, R, 1, 1, d, (uint64_t)R * d, (uint64_t)R * d);
+        ok &= make_map4(&maps.k4, a.kv_k0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
+        ok &= make_map4(&maps.v4, a.kv_v0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
+        if (!ok) {
+            L.status = QI21_ERR_CUDA;
+            return;
+        }
         gp.R = R;
         gp.m_blocks = (R + TC_BM - 1) / TC_BM;
         gp.M = a.M;
@@ -285,7 +323,22 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         }
         if (a.kv_only_last && l == c.n_layers - 1) break;
 
-        {
+        if (tc) {
+            AttnParams ap{};
+            ap.Mq = a.M;
+            ap.kv_len = a.kv_len;
+            ap.H = H;
+            ap.d = d;
+            ap.kv_limit = a.kv_limit;
+            ap.out = (bf16 *)a.o;
+            ap.scale_log2 = 1.4426950408889634f / sqrtf((float)Dh);
+            ap.layer = a.kv_layer_stride ? l : 0;
+            ap.err = a.err;
+            if (Dh == 128)
+                launch_attn_tc<128>(L, maps.q4, maps.k4, maps.v4, ap, a.B);
+            else
+                launch_attn_tc<64>(L, maps.q4, maps.k4, maps.v4, ap, a.B);
+        } else {
             const size_t smem = sizeof(float) * (3 * 32 * (Dh + 1) + 32 * 33);
             static bool attr_set = false;
             if (!attr_set) {
