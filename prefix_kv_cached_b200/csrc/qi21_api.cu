@@ -132,14 +132,29 @@ static int num_sms() {
 template <int EPI>
 static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, const CUtensorMap &b0,
                            const CUtensorMap &b1, const CUtensorMap &b2, const GemmParams &p) {
+    constexpr size_t smem = tc_smem_bytes<EPI>();
     static bool attr = false;
     if (!attr) {
-        cudaFuncSetAttribute(k_gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TC_SMEM_BYTES);
+        cudaFuncSetAttribute(k_gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         attr = true;
     }
     const int tiles = p.m_blocks * p.n_blocks;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, TC_SMEM_BYTES, L.st>>>(a, b0, b1, b2, p); });
+    L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
+}
+
+// 2-D fp32 tensor map [rows][inner] with a 32 x 32 box and 128-byte swizzle:
+// the target of the residual epilogue's TMA reduce-add.
+static bool make_map_f32(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows) {
+    if (!get_encode()) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 // 4-D bf16 tensor map [w][z][rows][inner] (strides in elements), box 64 x 128 x 1 x 1.
@@ -170,7 +185,7 @@ static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap 
 }
 
 struct TcMaps {
-    CUtensorMap xn, o, hid, wq, wk, wv, wo, wg, wu, wd, q4, k4, v4;
+    CUtensorMap xn, o, hid, wq, wk, wv, wo, wg, wu, wd, q4, k4, v4, h32;
 };
 
 static bool build_tc_maps(TcMaps &t, const qi21_config &c, const qi21_weights &w, const void *xn, const void *o,
@@ -267,6 +282,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         bool ok = make_map4(&maps.q4, a.q, d, R, 1, 1, d, (uint64_t)R * d, (uint64_t)R * d);
         ok &= make_map4(&maps.k4, a.kv_k0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
         ok &= make_map4(&maps.v4, a.kv_v0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
+        ok &= make_map_f32(&maps.h32, a.h, d, R);
         if (!ok) {
             L.status = QI21_ERR_CUDA;
             return;
@@ -357,7 +373,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             g.n_blocks = d / TC_BN;
             g.g_lo = tg1_lo;
             g.g_hi = tg1_hi;
-            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.wo, g);
+            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.h32, g);
         } else {
             launch_gemm_simt<T>(L, o, d, Wo, d, a.gemm, d, R, d, d);
             L.run("gated_residual", [&] {
@@ -376,7 +392,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             g2.n_blocks = d / TC_BN;
             g2.g_lo = tg2_lo;
             g2.g_hi = tg2_hi;
-            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.wd, g2);
+            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.h32, g2);
         } else {
             launch_gemm_simt<T>(L, xn, d, Wg, d, a.gemm, 2 * F, R, F, d);
             launch_gemm_simt<T>(L, xn, d, Wu, d, a.gemm + F, 2 * F, R, F, d);

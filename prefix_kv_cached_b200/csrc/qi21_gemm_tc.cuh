@@ -26,7 +26,14 @@ constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;          // 16 KB
 constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;          // 32 KB
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_THREADS = 192;
-constexpr size_t TC_SMEM_BYTES = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + 256;
+// EPI_RESIDUAL stages each epilogue warp's 32 x 32 fp32 box in shared memory
+// (two buffers per warp) for the TMA reduce-add into the residual stream.
+constexpr int TC_RED_BUF = 32 * 32 * 4;
+constexpr int TC_RED_BYTES = 4 * 2 * TC_RED_BUF;
+template <int EPI>
+constexpr size_t tc_smem_bytes() {
+    return 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + (EPI == EPI_RESIDUAL ? TC_RED_BYTES : 0) + 256;
+}
 
 struct GemmParams {
     int R;             // rows of A (tokens of all items)
@@ -58,6 +65,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&p);
 }
 
+// out[box] += smem box, element-wise in L2 (2-D fp32 tensor map, 128B swizzle).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *m, uint32_t src, int x, int y) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Store 32 fp32 values as bf16 (64 contiguous bytes, 16-byte aligned).
 __device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
@@ -87,7 +108,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *stage_base = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)TC_STAGES * TC_STAGE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)TC_STAGES * TC_STAGE_BYTES +
+                                                  (EPI == EPI_RESIDUAL ? TC_RED_BYTES : 0));
     uint64_t *full = bars, *empty = bars + TC_STAGES, *tfull = bars + 2 * TC_STAGES, *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -206,6 +228,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int quad = warp & 3;
         const int row_in_tile = quad * 32 + lane;
         int it = 0;
+        int red_count = 0;   // EPI_RESIDUAL: reduce-add boxes issued by this warp
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
             int m_blk, n_blk;
             tile_coords<EPI>(p, tile, m_blk, n_blk);
@@ -220,28 +243,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const int b = live ? r / p.M : 0;
             float v[32];
             if (EPI == EPI_RESIDUAL) {
+                // h[r][n] += tanh(gate)[n] * acc: each warp writes its 32 rows x 32 columns
+                // into a swizzled shared box and one lane reduce-adds the box into h.
                 const int n0 = n_blk * TC_BN;
                 const float *g = (m < p.split ? p.g_lo : p.g_hi) + n0;
-                float *hp = p.h + (size_t)r * p.ldh + n0;
+                uint8_t *stg = stage_base + (size_t)TC_STAGES * TC_STAGE_BYTES + (size_t)(warp - 2) * 2 * TC_RED_BUF;
+                const int sw = lane & 7;
 #pragma unroll 1
-                for (int cc = 0; cc < TC_BN / 32; ++cc) {
+                for (int cc = 0; cc < TC_BN / 32; ++cc, ++red_count) {
                     tmem_ld32(t_row + cc * 32, v);
                     tmem_wait_ld();
+                    if (cc == TC_BN / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(smem_u32(&tempty[acc]));
+                    }
                     if (live) {
-                        float4 *h4 = reinterpret_cast<float4 *>(hp + cc * 32);
                         const float4 *g4 = reinterpret_cast<const float4 *>(g + cc * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            float4 hv = h4[i];
                             const float4 gv = g4[i];
-                            hv.x = fmaf(gv.x, v[4 * i + 0], hv.x);
-                            hv.y = fmaf(gv.y, v[4 * i + 1], hv.y);
-                            hv.z = fmaf(gv.z, v[4 * i + 2], hv.z);
-                            hv.w = fmaf(gv.w, v[4 * i + 3], hv.w);
-                            h4[i] = hv;
+                            v[4 * i + 0] *= gv.x;
+                            v[4 * i + 1] *= gv.y;
+                            v[4 * i + 2] *= gv.z;
+                            v[4 * i + 3] *= gv.w;
                         }
                     }
+                    uint8_t *buf = stg + (red_count & 1) * TC_RED_BUF;
+                    if (red_count >= 2) {
+                        if (lane == 0) bulk_wait_group_read1();   // the reduce that used `buf` has read it
+                        __syncwarp();
+                    }
+                    uint8_t *rowp = buf + lane * 128;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4 *>(rowp + ((q ^ sw) << 4)) =
+                            make_float4(v[4 * q + 0], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_2d(&tmB2, smem_u32(buf), n0 + cc * 32, m_blk * TC_BM + quad * 32);
+                        bulk_commit_group();
+                    }
                 }
+                continue;   // TMEM already released
             } else if (EPI == EPI_SWIGLU) {
                 const int j0 = n_blk * 128;
                 float u[32];
@@ -312,6 +356,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
         }
+        if (EPI == EPI_RESIDUAL && lane == 0) bulk_wait_group0();
     }
     tc_fence_before();
     __syncthreads();
