@@ -48,7 +48,8 @@ enum {
     QI21_ERR_UNSUPPORTED = 5,      /* shape the selected kernel family does not cover */
     QI21_ERR_CUDA = 6,             /* a CUDA runtime / driver call failed */
     QI21_ERR_DEVICE_TIMEOUT = 7,   /* a bounded device wait expired */
-    QI21_ERR_WORKSPACE_TOO_SMALL = 8
+    QI21_ERR_WORKSPACE_TOO_SMALL = 8,
+    QI21_ERR_DEVICE_CHECK = 9      /* a kernel's own layout check failed; it returned without work */
 };
 
 /* Storage dtype of weights, activations and the K/V cache. The residual
@@ -249,7 +250,8 @@ qi21_status qi21_euler_update(const float *x_k, const float *v, double sigma_k, 
                               float *x_out, int64_t n, void *stream);
 
 /* Synchronise the stream, then read and clear the device error word of the
- * workspace. Returns QI21_OK, QI21_ERR_DEVICE_TIMEOUT or QI21_ERR_CUDA. */
+ * workspace. Returns QI21_OK, QI21_ERR_DEVICE_TIMEOUT, QI21_ERR_DEVICE_CHECK or
+ * QI21_ERR_CUDA. */
 qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *stream);
 
 const char *qi21_status_string(qi21_status s);

@@ -23,6 +23,7 @@ QI21_ERR_UNSUPPORTED = 5
 QI21_ERR_CUDA = 6
 QI21_ERR_DEVICE_TIMEOUT = 7
 QI21_ERR_WORKSPACE_TOO_SMALL = 8
+QI21_ERR_DEVICE_CHECK = 9
 
 QI21_DTYPE_F32 = 0
 QI21_DTYPE_BF16 = 1

@@ -687,7 +687,7 @@ extern "C" qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *
     if (word != 0) {
         if (cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return QI21_ERR_CUDA;
         cudaStreamSynchronize(st);
-        return QI21_ERR_DEVICE_TIMEOUT;
+        return word == DEV_ERR_TIMEOUT ? QI21_ERR_DEVICE_TIMEOUT : QI21_ERR_DEVICE_CHECK;
     }
     return QI21_OK;
 }

@@ -4,18 +4,27 @@
 // one of the kv_len keys (cached target rows: the target is last, so they see
 // the whole prefix cache and all target keys).
 //
-// One CTA per (item, head, 128 query rows); K/V tiles of 128 keys stream
-// through a 2-stage TMA ring (128-byte swizzle, no multicast).
-//   warp 0     : TMA producer (Q once, then K_j and V_j)
+// One CTA per (item, head, 128 query rows); K and V tiles of 128 keys stream
+// through two 2-stage TMA rings (128-byte swizzle, no multicast).
+//   warp 0     : TMA producers: lane 0 loads Q once, then K_j (a K stage is
+//                released as soon as its S MMA completes); lane 1 loads V_j (a
+//                V stage is released when its PV MMA completes)
 //   warp 1     : TMEM allocator + UMMA issuer:
-//                S_j = Q K_j^T  (M 128, N 128, K Dh)   -> TMEM S[j % 2]
-//                O_j = P_j V_j  (M 128, N Dh, K 128)  -> TMEM O[j % 2]
-//                P_j is read from shared memory (K-major), V_j as an MN-major operand.
-//   warps 2..5 : softmax, one query row per thread (TMEM lane): two passes over
-//                S_j (row max, then exp2 and the bf16 P row written swizzled to
-//                shared memory); O_{j-1} is folded into fp32 registers one tile
-//                late so that PV(j-1) runs under the softmax of tile j.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+Dh), O1 [384,384+Dh).
+//                S_j = Q K_j^T   (M 128, N 128, K Dh)  -> TMEM S[j % 2]
+//                O  += P_j V_j   (M 128, N Dh, K 128)  -> TMEM O (accumulated across tiles)
+//                P_j is read from shared memory (K-major, two buffers), V_j as an
+//                MN-major operand.
+//   warps 2..9 : softmax, two threads per query row (TMEM lane): warps w and
+//                w+4 share a lane quadrant and own key columns 0..63 / 64..127
+//                of S_j and the matching half of the O row. The halves swap
+//                their partial row max through shared memory behind a bounded
+//                mbarrier. The row keeps a running max m and only when a tile
+//                raises it by more than 2^8 (in the exp2 domain) do the two
+//                threads rescale their O halves in TMEM (after PV(j-1) has
+//                landed) — otherwise P_j = exp2(S_j c - m c) <= 256 is formed
+//                against the stale max, exactly as the final 1/l normalisation
+//                expects. S_{j+1} and PV(j-1) run under softmax(j).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dh).
 #pragma once
 #include "qi21_sm100.cuh"
 
@@ -63,33 +72,47 @@ struct AttnCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
-    static constexpr size_t SMEM = 1024 + (size_t)OFF_BAR + 256;
-    static constexpr int THREADS = 192;
+    static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;   // two P buffers
+    static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;       // [2][2 halves][128 rows] floats
+    static constexpr int OFF_BAR = OFF_RED + 2 * 2 * BQ * 4;
+    // The dynamic shared-memory window is checked to start on a 1024-byte
+    // boundary (the swizzled tiles need it), so no alignment slack is requested.
+    static constexpr size_t SMEM = (size_t)OFF_BAR + 256;
+    static constexpr int THREADS = 320;
+    static constexpr int SOFTMAX_THREADS = 256;
 };
 
+// Rescale the O row only when the running max grows by more than this (log2 units).
+constexpr float kRescaleLog2 = 8.0f;
+
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, AttnParams p) {
     using namespace sm100;
     using C = AttnCfg<DH>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    if (smem_u32(smem_raw) & 1023) {           // never expected; refuse rather than overrun
+        if (threadIdx.x == 0) raise_device_error(p.err, DEV_ERR_LAYOUT);
+        return;
+    }
+    uint8_t *smem = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars + 0;
     uint64_t *k_full = bars + 1;      // [2]
     uint64_t *v_full = bars + 3;      // [2]
-    uint64_t *kv_empty = bars + 5;    // [2]
+    uint64_t *k_empty = bars + 5;     // [2]  (S MMA of that K stage done)
     uint64_t *s_full = bars + 7;      // [2]
     uint64_t *s_empty = bars + 9;     // [2]
-    uint64_t *p_full = bars + 11;
-    uint64_t *o_full = bars + 12;     // [2]
-    uint64_t *o_empty = bars + 14;    // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    uint64_t *p_full = bars + 11;     // [2]
+    uint64_t *p_empty = bars + 13;    // [2]  (PV of that P buffer done)
+    uint64_t *xchg = bars + 15;       // [2]  (row-max halves exchanged)
+    uint64_t *lx = bars + 17;         //      (row-sum halves exchanged)
+    uint64_t *v_empty = bars + 18;    // [2]  (PV MMA of that V stage done)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *kv_end_s = reinterpret_cast<int *>(tmem_slot + 2);
+    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q0 = blockIdx.x * C::BQ, hh = blockIdx.y, b = blockIdx.z;
@@ -99,13 +122,15 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&k_full[i]), 1);
             mbar_init(smem_u32(&v_full[i]), 1);
-            mbar_init(smem_u32(&kv_empty[i]), 1);
+            mbar_init(smem_u32(&k_empty[i]), 1);
+            mbar_init(smem_u32(&v_empty[i]), 1);
             mbar_init(smem_u32(&s_full[i]), 1);
-            mbar_init(smem_u32(&s_empty[i]), 128);
-            mbar_init(smem_u32(&o_full[i]), 1);
-            mbar_init(smem_u32(&o_empty[i]), 128);
+            mbar_init(smem_u32(&s_empty[i]), C::SOFTMAX_THREADS);
+            mbar_init(smem_u32(&p_full[i]), C::SOFTMAX_THREADS);
+            mbar_init(smem_u32(&p_empty[i]), 1);
+            mbar_init(smem_u32(&xchg[i]), C::SOFTMAX_THREADS);
         }
-        mbar_init(smem_u32(p_full), 128);
+        mbar_init(smem_u32(lx), C::SOFTMAX_THREADS);
         *abort_flag = 0;
         *kv_end_s = 0;
         fence_barrier_init();
@@ -118,7 +143,7 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     // keys this CTA needs: the largest limit over its query rows
-    if (threadIdx.x >= 64) {
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + C::BQ) {
         const int row = q0 + (threadIdx.x - 64);
         int lim = 0;
         if (row < p.Mq) lim = p.kv_limit ? min(p.kv_limit[row], p.kv_len) : p.kv_len;
@@ -130,8 +155,10 @@ __global__ void __launch_bounds__(192, 1)
     const int T = (kv_end + C::BK - 1) / C::BK;
 
     if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producers
+        // lane 0 streams K (a stage frees as soon as its S MMA is done, so K runs
+        // two tiles ahead); lane 1 streams V (a stage frees after its PV MMA).
         if (lane == 0 && T > 0) {
-            // ------------------------------------------------------------ TMA producer
             const uint32_t qb = smem_u32(q_full);
             mbar_arrive_expect_tx(qb, C::Q_BYTES);
             for (int x = 0; x < C::BOXES; ++x)
@@ -139,12 +166,18 @@ __global__ void __launch_bounds__(192, 1)
                             b * p.Mq + q0, 0, 0);
             for (int j = 0; j < T; ++j) {
                 const int s = j & 1;
-                if (!mbar_wait(smem_u32(&kv_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-                const uint32_t kb = smem_u32(&k_full[s]), vb = smem_u32(&v_full[s]);
+                if (!mbar_wait(smem_u32(&k_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+                const uint32_t kb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(kb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
                     tma_load_4d(smem_u32(smem + C::OFF_K + s * C::KV_BYTES + x * (C::BK * 128)), &tmK, kb,
                                 hh * DH + x * 64, j * C::BK, b, p.layer);
+            }
+        } else if (lane == 1 && T > 0) {
+            for (int j = 0; j < T; ++j) {
+                const int s = j & 1;
+                if (!mbar_wait(smem_u32(&v_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+                const uint32_t vb = smem_u32(&v_full[s]);
                 mbar_arrive_expect_tx(vb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
                     tma_load_4d(smem_u32(smem + C::OFF_V + s * C::KV_BYTES + x * (C::BK * 128)), &tmV, vb,
@@ -157,41 +190,41 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t idesc_s = idesc_bf16_f32(C::BQ, C::BK);
             constexpr uint32_t idesc_o = idesc_bf16_f32(C::BQ, DH, true);
             const uint32_t sq = smem_u32(smem + C::OFF_Q);
-            const uint32_t sp = smem_u32(smem + C::OFF_P);
+            const uint32_t o_tmem = tmem_base + 256;
             bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.err);
-            auto issue_pv = [&](int jj) -> bool {
-                const int s = jj & 1, ob = jj & 1;
-                if (!mbar_wait(smem_u32(p_full), jj & 1, abort_flag, p.err)) return false;
-                if (!mbar_wait(smem_u32(&v_full[s]), (jj >> 1) & 1, abort_flag, p.err)) return false;
-                if (!mbar_wait(smem_u32(&o_empty[ob]), ((jj >> 1) & 1) ^ 1, abort_flag, p.err)) return false;
+            auto issue_pv = [&](int i) -> bool {
+                const int s = i & 1;
+                if (!mbar_wait(smem_u32(&p_full[s]), (i >> 1) & 1, abort_flag, p.err)) return false;
+                if (!mbar_wait(smem_u32(&v_full[s]), (i >> 1) & 1, abort_flag, p.err)) return false;
                 tc_fence_after();
+                const uint32_t sp = smem_u32(smem + C::OFF_P + s * C::P_BYTES);
                 const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
-                const uint32_t d_tmem = tmem_base + 256 + ob * 128;
 #pragma unroll
                 for (int k = 0; k < C::BK / 16; ++k) {
                     const uint64_t adesc = sdesc_kmajor_sw128(sp + (k >> 2) * (C::BQ * 128) + (k & 3) * 32);
                     const uint64_t bdesc = sdesc_mnmajor_sw128(sv + k * 2048, C::BK * 128);
-                    umma_f16(d_tmem, adesc, bdesc, idesc_o, k > 0 ? 1u : 0u);
+                    umma_f16(o_tmem, adesc, bdesc, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
                 }
-                umma_commit(smem_u32(&o_full[ob]));
-                umma_commit(smem_u32(&kv_empty[s]));
+                umma_commit(smem_u32(&p_empty[s]));
+                umma_commit(smem_u32(&v_empty[s]));
                 return true;
             };
             for (int j = 0; j < T && ok; ++j) {
-                const int s = j & 1, sb = j & 1;
+                const int s = j & 1;
                 if (!mbar_wait(smem_u32(&k_full[s]), (j >> 1) & 1, abort_flag, p.err)) break;
-                if (!mbar_wait(smem_u32(&s_empty[sb]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+                if (!mbar_wait(smem_u32(&s_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KV_BYTES);
-                const uint32_t d_tmem = tmem_base + sb * 128;
+                const uint32_t d_tmem = tmem_base + s * 128;
 #pragma unroll
                 for (int k = 0; k < DH / 16; ++k) {
                     const uint32_t off = (k >> 2) * (C::BQ * 128) + (k & 3) * 32;
-                    umma_f16(d_tmem, sdesc_kmajor_sw128(sq + off), sdesc_kmajor_sw128(sk + (k >> 2) * (C::BK * 128) +
-                                                                                     (k & 3) * 32),
-                             idesc_s, k > 0 ? 1u : 0u);
+                    umma_f16(d_tmem, sdesc_kmajor_sw128(sq + off),
+                             sdesc_kmajor_sw128(sk + (k >> 2) * (C::BK * 128) + (k & 3) * 32), idesc_s,
+                             k > 0 ? 1u : 0u);
                 }
-                umma_commit(smem_u32(&s_full[sb]));
+                umma_commit(smem_u32(&s_full[s]));
+                umma_commit(smem_u32(&k_empty[s]));
                 if (j >= 1 && !issue_pv(j - 1)) {
                     ok = false;
                     break;
@@ -200,133 +233,134 @@ __global__ void __launch_bounds__(192, 1)
             if (ok) issue_pv(T - 1);
         }
     } else {
-        // ---------------------------------------------------------------- softmax warps
+        // ---------------------------------------------------------------- softmax warps (2..9)
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;                // key columns half*64 .. +63, O columns half*DH/2 ..
         const int r = quad * 32 + lane;                  // row within the tile = TMEM lane
         const int row = q0 + r;
         int lim = p.kv_len;
         if (p.kv_limit && row < p.Mq) lim = min(p.kv_limit[row], p.kv_len);
         const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-        uint8_t *prow = smem + C::OFF_P + r * 128;       // row r of each 64-key box
+        const uint32_t t_o = t_lane + 256 + half * (DH / 2);
         const int sw = r & 7;
-        float o[DH];
-#pragma unroll
-        for (int i = 0; i < DH; ++i) o[i] = 0.f;
-        float m_run = -INFINITY, l_run = 0.f, alpha_prev = 0.f;
         const float c = p.scale_log2;
+        float m_run = -INFINITY, l_half = 0.f;
         bool ok = true;
-        float v[32];
+        float sv[64];
+        // tcgen05.ld / tcgen05.st are warp-collective (.sync.aligned): every
+        // decision that guards one is made uniform across the warp.
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag, p.err) ? 1 : 0) != 0;
+        };
         for (int j = 0; j < T && ok; ++j) {
-            const int sb = j & 1;
-            if (!mbar_wait(smem_u32(&s_full[sb]), (j >> 1) & 1, abort_flag, p.err)) {
+            const int s = j & 1;
+            if (!wait_all(&s_full[s], (j >> 1) & 1)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int key0 = j * C::BK;
-            // pass 1: row max over the allowed keys
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                tmem_ld32(t_lane + sb * 128 + cc * 32, v);
-                tmem_wait_ld();
-                const int kb = key0 + cc * 32;
-                if (kb + 32 <= lim) {
+            tmem_ld32(t_lane + s * 128 + half * 64, *reinterpret_cast<float(*)[32]>(&sv[0]));
+            tmem_ld32(t_lane + s * 128 + half * 64 + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&s_empty[s]));
+            const int key0 = j * C::BK + half * 64;
+            if (key0 + 64 > lim) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, v[i]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (kb + i < lim) mx = fmaxf(mx, v[i]);
-                }
+                for (int i = 0; i < 64; ++i)
+                    if (key0 + i >= lim) sv[i] = -INFINITY;
             }
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha = (m_new == -INFINITY) ? 1.f : ex2_approx((m_run - m_new) * c);
-            const float mc = (m_new == -INFINITY) ? 0.f : m_new * c;
-            // P buffer is free once PV(j-1) finished; O_{j-1} is then ready too
-            if (j >= 1) {
-                if (!mbar_wait(smem_u32(&o_full[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort_flag, p.err)) {
+            float m8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m8[i] = sv[i];
+#pragma unroll
+            for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
+            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            // swap the half-row maxima
+            float *red_j = red + (s * 2) * C::BQ;
+            red_j[half * C::BQ + r] = mx;
+            mbar_arrive(smem_u32(&xchg[s]));
+            if (!wait_all(&xchg[s], (j >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, red_j[(half ^ 1) * C::BQ + r]);
+            // per row: move the running max only when this tile raises it by more than 2^8
+            const bool first = (m_run == -INFINITY);
+            const bool grow = first || (mx - m_run) * c > kRescaleLog2;
+            const float m_new = grow ? fmaxf(m_run, mx) : m_run;
+            const float alpha = (grow && !first) ? ex2_approx((m_run - m_new) * c) : 1.f;
+            if (__any_sync(0xffffffffu, grow && !first)) {
+                // O holds PV(0..j-1) against the old max: the whole warp rescales its
+                // O rows (alpha = 1 where the row's max did not move) once PV(j-1) landed
+                if (!wait_all(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-            }
-            // pass 2: p = exp2(s c - m c), bf16 P row into shared memory (128B swizzle)
-            float rs = 0.f;
-#pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                tmem_ld32(t_lane + sb * 128 + cc * 32, v);
-                tmem_wait_ld();
-                const int kb = key0 + cc * 32;
-                if (kb + 32 <= lim) {
+                float ov[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        v[i] = ex2_approx(fmaf(v[i], c, -mc));
-                        rs += v[i];
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        v[i] = (kb + i < lim) ? ex2_approx(fmaf(v[i], c, -mc)) : 0.f;
-                        rs += v[i];
-                    }
-                }
-                // keys cc*32 .. cc*32+31 live in box cc/2, 16-byte chunks (cc%2)*4 .. +3
-                uint8_t *box = prow + (cc >> 1) * (C::BQ * 128);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = (cc & 1) * 4 + q;
-                    uint4 u;
-                    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-                    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-                    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-                    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-                    *reinterpret_cast<uint4 *>(box + ((chunk ^ sw) << 4)) = u;
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&s_empty[sb]));
-            fence_proxy_async_smem();
-            mbar_arrive(smem_u32(p_full));
-            l_run = l_run * alpha + rs;
-            m_run = m_new;
-            // fold O_{j-1} (scale m_{j-1}) into o (scale m_{j-2})
-            if (j >= 1) {
-                const int ob = (j - 1) & 1;
-#pragma unroll
-                for (int cc = 0; cc < DH / 32; ++cc) {
-                    tmem_ld32(t_lane + 256 + ob * 128 + cc * 32, v);
+                for (int cc = 0; cc < DH / 64; ++cc) {
+                    tmem_ld32(t_o + cc * 32, ov);
                     tmem_wait_ld();
+                    uint32_t u[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[cc * 32 + i] = fmaf(o[cc * 32 + i], alpha_prev, v[i]);
+                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(ov[i] * alpha);
+                    tmem_st32(t_o + cc * 32, u);
                 }
-                tc_fence_before();
-                mbar_arrive(smem_u32(&o_empty[ob]));
+                tmem_wait_st();
             }
-            alpha_prev = alpha;
+            l_half *= alpha;
+            m_run = m_new;
+            const float mc = m_run * c;
+            float s8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s8[i] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                sv[i] = ex2_approx(fmaf(sv[i], c, -mc));    // masked: exp2(-inf) = 0
+                s8[i & 7] += sv[i];
+            }
+            l_half += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+            // P buffer s is free once PV(j-2) has completed
+            if (!wait_all(&p_empty[s], ((j >> 1) & 1) ^ 1)) {
+                ok = false;
+                break;
+            }
+            // this half's 64 keys form one 128-byte swizzled box row
+            uint8_t *prow = smem + C::OFF_P + s * C::P_BYTES + half * (C::BQ * 128) + r * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float *v8 = &sv[8 * q];
+                uint4 u;
+                u.x = pack_bf16x2(v8[0], v8[1]);
+                u.y = pack_bf16x2(v8[2], v8[3]);
+                u.z = pack_bf16x2(v8[4], v8[5]);
+                u.w = pack_bf16x2(v8[6], v8[7]);
+                *reinterpret_cast<uint4 *>(prow + ((q ^ sw) << 4)) = u;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&p_full[s]));
         }
         if (ok && T > 0) {
-            const int ob = (T - 1) & 1;
-            if (mbar_wait(smem_u32(&o_full[ob]), ((T - 1) >> 1) & 1, abort_flag, p.err)) {
+            // combine the half-row sums (the buffer of tile T is free: its readers finished at T-1)
+            float *red_l = red + ((T & 1) * 2) * C::BQ;
+            red_l[half * C::BQ + r] = l_half;
+            mbar_arrive(smem_u32(lx));
+            if (wait_all(lx, 0) && wait_all(&p_empty[(T - 1) & 1], ((T - 1) >> 1) & 1)) {
                 tc_fence_after();
+                const float inv = 1.f / (l_half + red_l[(half ^ 1) * C::BQ + r]);
+                bf16 *dst = p.out + ((size_t)b * p.Mq + row) * p.d + hh * DH + half * (DH / 2);
+                float ov[32];
 #pragma unroll
-                for (int cc = 0; cc < DH / 32; ++cc) {
-                    tmem_ld32(t_lane + 256 + ob * 128 + cc * 32, v);
+                for (int cc = 0; cc < DH / 64; ++cc) {
+                    tmem_ld32(t_o + cc * 32, ov);          // every lane: the load is warp-collective
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[cc * 32 + i] = fmaf(o[cc * 32 + i], alpha_prev, v[i]);
-                }
-                tc_fence_before();
-                mbar_arrive(smem_u32(&o_empty[ob]));
-                if (row < p.Mq) {
-                    const float inv = 1.f / l_run;
-                    bf16 *dst = p.out + ((size_t)b * p.Mq + row) * p.d + hh * DH;
-#pragma unroll
-                    for (int cc = 0; cc < DH / 32; ++cc) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = o[cc * 32 + i] * inv;
-                        store_bf16x32(dst + cc * 32, v);
-                    }
+                    for (int i = 0; i < 32; ++i) ov[i] *= inv;
+                    if (row < p.Mq) store_bf16x32(dst + cc * 32, ov);
                 }
             }
         }

@@ -45,7 +45,7 @@ __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x));
 
 // Error word in the workspace: kernels set a code and return instead of
 // trapping; the host reads it with qi21_check_device_error.
-enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1 };
+enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_LAYOUT = 2 };
 
 __device__ __forceinline__ void raise_device_error(uint32_t *err, uint32_t code) {
     if (err) atomicCAS(err, 0u, code);

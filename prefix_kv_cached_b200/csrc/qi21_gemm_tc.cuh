@@ -234,7 +234,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tile_coords<EPI>(p, tile, m_blk, n_blk);
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.err)) break;
+            // warp-uniform: the tcgen05.ld below is warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.err) ? 1 : 0))
+                break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * TC_BN);
             const int r = m_blk * TC_BM + row_in_tile;

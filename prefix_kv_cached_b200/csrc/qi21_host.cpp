@@ -117,6 +117,7 @@ extern "C" const char *qi21_status_string(qi21_status s) {
         case QI21_ERR_CUDA: return "CUDA error";
         case QI21_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case QI21_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case QI21_ERR_DEVICE_CHECK: return "a kernel's device-side layout check failed";
         default: return "unknown status";
     }
 }
