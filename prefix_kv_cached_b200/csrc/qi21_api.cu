@@ -138,7 +138,7 @@ static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, 
         cudaFuncSetAttribute(k_gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         attr = true;
     }
-    const int tiles = p.m_blocks * p.n_blocks;
+    const int tiles = p.m_blocks * p.n_blocks * p.ksplit;
     const int grid = tiles < num_sms() ? tiles : num_sms();
     L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
 }
@@ -182,6 +182,16 @@ static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap 
     }
     dim3 grid((p.Mq + Cf::BQ - 1) / Cf::BQ, p.H, B);
     L.run("attn", [&] { k_attn_tc<DH><<<grid, Cf::THREADS, Cf::SMEM, L.st>>>(q, k, v, p); });
+}
+
+// K slices for a residual GEMM: enough work units for about six waves of the
+// persistent grid (the reduce-add epilogue sums the slices in L2), at least
+// eight K blocks per slice.
+static int residual_ksplit(int tiles, int kblocks) {
+    const int target = 6 * num_sms();
+    int ks = 1;
+    while (ks < 4 && tiles * ks < target && kblocks / (ks + 1) >= 8) ++ks;
+    return ks;
 }
 
 struct TcMaps {
@@ -289,6 +299,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         }
         gp.R = R;
         gp.m_blocks = (R + TC_BM - 1) / TC_BM;
+        gp.ksplit = 1;
         gp.M = a.M;
         gp.split = a.split;
         gp.h = a.h;
@@ -371,6 +382,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             GemmParams g = gp;
             g.K = d;
             g.n_blocks = d / TC_BN;
+            g.ksplit = residual_ksplit(g.m_blocks * g.n_blocks, d / TC_BK);
             g.g_lo = tg1_lo;
             g.g_hi = tg1_hi;
             launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.h32, g);
@@ -390,6 +402,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             GemmParams g2 = gp;
             g2.K = F;
             g2.n_blocks = d / TC_BN;
+            g2.ksplit = residual_ksplit(g2.m_blocks * g2.n_blocks, F / TC_BK);
             g2.g_lo = tg2_lo;
             g2.g_hi = tg2_hi;
             launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.h32, g2);

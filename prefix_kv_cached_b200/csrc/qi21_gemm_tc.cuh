@@ -40,6 +40,7 @@ struct GemmParams {
     int K;             // reduction length
     int m_blocks;      // ceil(R / 128)
     int n_blocks;      // output tiles along N
+    int ksplit;        // EPI_RESIDUAL: K slices per output tile, each reduce-added into h (1 otherwise)
     int M, split;      // rows per item; rows m < split read the prefix modulation row
     // EPI_RESIDUAL
     float *h;
@@ -93,11 +94,18 @@ __device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
     }
 }
 
-template <int EPI>
-__device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int &m_blk, int &n_blk) {
-    // m fastest: CTAs running together share a weight tile, activations stay in L2
+// Work unit -> (row block, column block, K slice). m fastest: CTAs running
+// together share a weight tile while the activations stay in L2. With
+// ksplit > 1 (residual epilogue only) a unit covers K blocks [kb0, kb1); its
+// partial product is reduce-added into h like a whole tile's.
+__device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int kblocks, int &m_blk, int &n_blk,
+                                            int &kb0, int &kb1) {
     m_blk = tile % p.m_blocks;
-    n_blk = tile / p.m_blocks;
+    const int rest = tile / p.m_blocks;
+    n_blk = rest % p.n_blocks;
+    const int ks = rest / p.n_blocks;
+    kb0 = (int)((int64_t)kblocks * ks / p.ksplit);
+    kb1 = (int)((int64_t)kblocks * (ks + 1) / p.ksplit);
 }
 
 template <int EPI>
@@ -115,7 +123,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = p.m_blocks * p.n_blocks;
+    const int num_tiles = p.m_blocks * p.n_blocks * p.ksplit;
     const int kblocks = p.K / TC_BK;
 
     if (threadIdx.x == 0) {
@@ -152,8 +160,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                int m_blk, n_blk;
-                tile_coords<EPI>(p, tile, m_blk, n_blk);
+                int m_blk, n_blk, kb0, kb1;
+                tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
                 const CUtensorMap *b0 = &tmB0, *b1 = &tmB1;
                 int rb0, rb1;
                 if (EPI == EPI_SWIGLU) {
@@ -168,7 +176,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     rb0 = n_blk * TC_BN;
                     rb1 = rb0 + 128;
                 }
-                for (int kb = 0; kb < kblocks; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.err)) {
                         ok = false;
                         break;
@@ -196,12 +204,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             int it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+                int m_blk, n_blk, kb0, kb1;
+                tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
-                for (int kb = 0; kb < kblocks; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.err)) {
                         ok = false;
                         break;
@@ -212,7 +222,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < TC_BK / 16; ++k) {
                         umma_f16(d_tmem, sdesc_kmajor_sw128(sa + k * 32), sdesc_kmajor_sw128(sb + k * 32), idesc,
-                                 (kb > 0 || k > 0) ? 1u : 0u);
+                                 (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(smem_u32(&empty[stage]));
                     if (++stage == TC_STAGES) {
@@ -230,8 +240,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         int it = 0;
         int red_count = 0;   // EPI_RESIDUAL: reduce-add boxes issued by this warp
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-            int m_blk, n_blk;
-            tile_coords<EPI>(p, tile, m_blk, n_blk);
+            int m_blk, n_blk, kb0, kb1;
+            tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             // warp-uniform: the tcgen05.ld below is warp-collective
