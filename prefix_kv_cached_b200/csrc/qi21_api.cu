@@ -426,6 +426,12 @@ static void launch_img_in(Launcher &L, const qi21_config &c, const float *x, con
                           int N, int M_out, int off) {
     const int rows = B * N, C = c.latent_ch, d = c.d_model;
     dim3 grid((rows + 15) / 16, (d + 255) / 256);
+    if (C == 64) {
+        L.run("img_in", [&] {
+            k_img_in64<T><<<grid, 256, 0, L.st>>>(x, (const T *)w_img_in, h, rows, d, N, M_out, off);
+        });
+        return;
+    }
     L.run("img_in", [&] {
         k_img_in<T><<<grid, 256, sizeof(float) * 16 * C, L.st>>>(x, (const T *)w_img_in, h, rows, C, d, N, M_out, off);
     });
@@ -435,6 +441,12 @@ template <typename T>
 static void launch_final(Launcher &L, const qi21_config &c, const float *h, int M, int off, int B, int N,
                          const float *sf, const void *w_out, float *v) {
     const int rows = B * N, d = c.d_model;
+    if (c.latent_ch == 64 && d % 128 == 0) {
+        L.run("final", [&] {
+            k_final64<T><<<(rows + 15) / 16, 256, 0, L.st>>>(h, M, off, N, d, sf, (const T *)w_out, c.ln_eps, v, rows);
+        });
+        return;
+    }
     const size_t smem = sizeof(float) * 4 * d;
     static bool attr_set[2] = {false, false};
     if (smem > 48 * 1024 && !attr_set[sizeof(T) == 2]) {

@@ -154,6 +154,61 @@ __global__ void __launch_bounds__(256) k_img_in(const float *__restrict__ x, con
     }
 }
 
+// img_in for 64 latent channels: each thread keeps its output column's 64
+// weights in registers (eight 16-byte loads) and produces 16 rows.
+template <typename T>
+__global__ void __launch_bounds__(256) k_img_in64(const float *__restrict__ x, const T *__restrict__ W,
+                                                  float *__restrict__ h, int rows, int d, int N, int M_out, int off) {
+    constexpr int C = 64;
+    __shared__ float xs[16][C];
+    const int r0 = blockIdx.x * 16;
+    for (int e = threadIdx.x; e < 16 * C; e += blockDim.x) {
+        const int i = e / C, k = e % C;
+        xs[i][k] = (r0 + i < rows) ? x[(size_t)(r0 + i) * C + k] : 0.f;
+    }
+    const int c = blockIdx.y * 256 + threadIdx.x;
+    float w[C];
+    if (c < d) {
+        if constexpr (sizeof(T) == 2) {
+            const uint4 *w8 = reinterpret_cast<const uint4 *>(W + (size_t)c * C);
+#pragma unroll
+            for (int q = 0; q < C / 8; ++q) {
+                const uint4 u = w8[q];
+                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = __bfloat1622float2(p2[t]);
+                    w[8 * q + 2 * t] = f.x;
+                    w[8 * q + 2 * t + 1] = f.y;
+                }
+            }
+        } else {
+            const float4 *w4 = reinterpret_cast<const float4 *>(W + (size_t)c * C);
+#pragma unroll
+            for (int q = 0; q < C / 4; ++q) {
+                const float4 f = w4[q];
+                w[4 * q] = f.x;
+                w[4 * q + 1] = f.y;
+                w[4 * q + 2] = f.z;
+                w[4 * q + 3] = f.w;
+            }
+        }
+    }
+    __syncthreads();
+    if (c >= d) return;
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int r = r0 + i;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < C; ++k) acc = fmaf(xs[i][k], w[k], acc);
+        if (r < rows) {
+            const int b = r / N, n = r % N;
+            h[((size_t)b * M_out + off + n) * d + c] = acc;
+        }
+    }
+}
+
 // Copy the prefix hidden states [B][P][d] into residual rows b*M_out + n.
 static __global__ void k_copy_rows(const float *__restrict__ src, float *__restrict__ dst, int rows_per_item, int d,
                             int M_out, int64_t total) {
@@ -428,6 +483,80 @@ __global__ void __launch_bounds__(256) k_final(const float *__restrict__ h, int 
         for (int k = lane; k < d; k += 32) acc = fmaf(xs[i * d + k], to_f(w[k]), acc);
         acc = warp_sum(acc);
         if (lane == 0 && r0 + i < rows) v[(size_t)(r0 + i) * C + c] = acc;
+    }
+}
+
+// Final AdaLN + proj_out for 64 latent channels and d % 128 == 0, tiled:
+// 16 rows x 64 outputs per block. Row statistics first (one warp per two
+// rows, two-pass), then K chunks of 128: the normalised, scaled rows and the
+// matching W_out columns are staged in shared memory and each thread
+// accumulates one row x four outputs.
+template <typename T>
+__global__ void __launch_bounds__(256) k_final64(const float *__restrict__ h, int M, int off, int N, int d,
+                                                 const float *__restrict__ sf, const T *__restrict__ Wout, float eps,
+                                                 float *__restrict__ v, int rows) {
+    constexpr int RB = 16, C = 64, KC = 128;
+    __shared__ float mean_s[RB], rstd_s[RB];
+    __shared__ float xs[RB][KC];
+    __shared__ float ws[C][KC + 1];
+    const int r0 = blockIdx.x * RB;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int i = wid; i < RB; i += 8) {
+        const int r = r0 + i;
+        float mean = 0.f, rstd = 0.f;
+        if (r < rows) {
+            const int b = r / N, n = r % N;
+            const float4 *x4 = reinterpret_cast<const float4 *>(h + ((size_t)b * M + off + n) * d);
+            float s = 0.f;
+            for (int c4 = lane; c4 < d / 4; c4 += 32) {
+                const float4 a = x4[c4];
+                s += (a.x + a.y) + (a.z + a.w);
+            }
+            mean = warp_sum(s) / d;
+            float q = 0.f;
+            for (int c4 = lane; c4 < d / 4; c4 += 32) {
+                const float4 a = x4[c4];
+                const float e0 = a.x - mean, e1 = a.y - mean, e2 = a.z - mean, e3 = a.w - mean;
+                q += (e0 * e0 + e1 * e1) + (e2 * e2 + e3 * e3);
+            }
+            rstd = 1.0f / sqrtf(warp_sum(q) / d + eps);
+        }
+        if (lane == 0) {
+            mean_s[i] = mean;
+            rstd_s[i] = rstd;
+        }
+    }
+    __syncthreads();
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;     // row ty, outputs 4tx .. 4tx+3
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k0 = 0; k0 < d; k0 += KC) {
+        for (int e = threadIdx.x; e < RB * KC; e += 256) {
+            const int i = e / KC, k = e % KC;
+            const int r = r0 + i;
+            float val = 0.f;
+            if (r < rows) {
+                const int b = r / N, n = r % N;
+                val = (h[((size_t)b * M + off + n) * d + k0 + k] - mean_s[i]) * rstd_s[i] * (1.f + sf[k0 + k]);
+            }
+            xs[i][k] = val;
+        }
+        for (int e = threadIdx.x; e < C * KC; e += 256) {
+            const int cc = e / KC, k = e % KC;
+            ws[cc][k] = to_f(Wout[(size_t)cc * d + k0 + k]);
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < KC; ++k) {
+            const float xv = xs[ty][k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[j] = fmaf(xv, ws[4 * tx + j][k], acc[j]);
+        }
+        __syncthreads();
+    }
+    const int r = r0 + ty;
+    if (r < rows) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[(size_t)r * C + 4 * tx + j] = acc[j];
     }
 }
 
