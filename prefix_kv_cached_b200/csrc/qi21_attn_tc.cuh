@@ -12,7 +12,7 @@
 //   warp 1     : TMEM allocator + UMMA issuer:
 //                S_j = Q K_j^T   (M 128, N 128, K Dh)  -> TMEM S[j % 2]
 //                O  += P_j V_j   (M 128, N Dh, K 128)  -> TMEM O (accumulated across tiles)
-//                P_j is read from shared memory (K-major, two buffers), V_j as an
+//                P_j (bf16) is read from TMEM, V_j from shared memory as an
 //                MN-major operand.
 //   warps 2..9 : softmax, two threads per query row (TMEM lane): warps w and
 //                w+4 share a lane quadrant and own key columns 0..63 / 64..127
@@ -24,7 +24,8 @@
 //                landed) — otherwise P_j = exp2(S_j c - m c) <= 256 is formed
 //                against the stale max, exactly as the final 1/l normalisation
 //                expects. S_{j+1} and PV(j-1) run under softmax(j).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+Dh).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+Dh), P0 [384,448),
+// P1 [448,512) (P rows as bf16 pairs: key k of row r at lane r, column k/2).
 #pragma once
 #include "qi21_sm100.cuh"
 
@@ -67,13 +68,11 @@ struct AttnCfg {
     static constexpr int BOXES = DH / 64;                  // 64-element (128-byte) swizzle boxes per row
     static constexpr int Q_BYTES = BQ * DH * 2;
     static constexpr int KV_BYTES = BK * DH * 2;           // one K or V tile
-    static constexpr int P_BYTES = BQ * BK * 2;            // 32 KB
     static constexpr int STAGES = 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;   // two P buffers
-    static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;       // [2][2 halves][128 rows] floats
+    static constexpr int OFF_RED = OFF_V + STAGES * KV_BYTES;  // [2][2 halves][128 rows] floats
     static constexpr int OFF_BAR = OFF_RED + 2 * 2 * BQ * 4;
     // The dynamic shared-memory window is checked to start on a 1024-byte
     // boundary (the swizzled tiles need it), so no alignment slack is requested.
@@ -197,13 +196,12 @@ __global__ void __launch_bounds__(320, 1)
                 if (!mbar_wait(smem_u32(&p_full[s]), (i >> 1) & 1, abort_flag, p.err)) return false;
                 if (!mbar_wait(smem_u32(&v_full[s]), (i >> 1) & 1, abort_flag, p.err)) return false;
                 tc_fence_after();
-                const uint32_t sp = smem_u32(smem + C::OFF_P + s * C::P_BYTES);
+                const uint32_t p_tmem = tmem_base + 384 + s * 64;
                 const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
                 for (int k = 0; k < C::BK / 16; ++k) {
-                    const uint64_t adesc = sdesc_kmajor_sw128(sp + (k >> 2) * (C::BQ * 128) + (k & 3) * 32);
                     const uint64_t bdesc = sdesc_mnmajor_sw128(sv + k * 2048, C::BK * 128);
-                    umma_f16(o_tmem, adesc, bdesc, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
+                    umma_f16_ts(o_tmem, p_tmem + k * 8, bdesc, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
                 }
                 umma_commit(smem_u32(&p_empty[s]));
                 umma_commit(smem_u32(&v_empty[s]));
@@ -242,7 +240,6 @@ __global__ void __launch_bounds__(320, 1)
         if (p.kv_limit && row < p.Mq) lim = min(p.kv_limit[row], p.kv_len);
         const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
         const uint32_t t_o = t_lane + 256 + half * (DH / 2);
-        const int sw = r & 7;
         const float c = p.scale_log2;
         float m_run = -INFINITY, l_half = 0.f;
         bool ok = true;
@@ -328,19 +325,14 @@ __global__ void __launch_bounds__(320, 1)
                 ok = false;
                 break;
             }
-            // this half's 64 keys form one 128-byte swizzled box row
-            uint8_t *prow = smem + C::OFF_P + s * C::P_BYTES + half * (C::BQ * 128) + r * 128;
+            // this half's 64 keys -> 32 TMEM columns of P[s] (bf16 pairs, lower key in the low half)
+            {
+                uint32_t u[32];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float *v8 = &sv[8 * q];
-                uint4 u;
-                u.x = pack_bf16x2(v8[0], v8[1]);
-                u.y = pack_bf16x2(v8[2], v8[3]);
-                u.z = pack_bf16x2(v8[4], v8[5]);
-                u.w = pack_bf16x2(v8[6], v8[7]);
-                *reinterpret_cast<uint4 *>(prow + ((q ^ sw) << 4)) = u;
+                for (int q = 0; q < 32; ++q) u[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
+                tmem_st32(t_lane + 384 + s * 64 + half * 32, u);
+                tmem_wait_st();
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(smem_u32(&p_full[s]));
         }
