@@ -240,6 +240,13 @@ def dist_barrier(world: int):
         dist.barrier()
 
 
+def aggregate(world: int, tokens_per_rank: int, steps: int, ms_local: float):
+    """Whole-job throughput of independent replicas: every rank processed
+    tokens_per_rank * steps tokens; the job took the slowest rank's time."""
+    ms_max = dist_max(ms_local, world)
+    return ms_max, world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 def dist_done(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -361,11 +368,10 @@ def main():
     B.qi21_profile_enable(0)
     prof = B.qi21_profile_read()
     ms = t0.elapsed_time(t1)
-    ms_max = dist_max(ms, world)
+    tokens = w.batch * w.n_target
+    ms_max, value = aggregate(world, tokens, args.steps, ms)
     r.check_device()
     ms_step = ms_max / args.steps
-    tokens = w.batch * w.n_target
-    value = world * tokens * args.steps / (ms_max / 1e3)
 
     # e2e: same step through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None

@@ -256,6 +256,14 @@ qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *stream);
 
 const char *qi21_status_string(qi21_status s);
 
+/* Self test of the failure path (not part of the pages' method): launches a
+ * kernel whose single bounded wait can never be satisfied, with a limit of
+ * limit_ns nanoseconds (1 .. 10^9). The wait gives up, sets the workspace's
+ * device error word and the kernel returns normally, so
+ * qi21_check_device_error must then report QI21_ERR_DEVICE_TIMEOUT (and clear
+ * the word). Nothing traps, faults or hangs. */
+qi21_status qi21_selftest_wait_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream);
+
 /* ---------------------------------------------------------------- per-kernel timing */
 
 /* When enabled, the entry points record a CUDA event pair on their stream

@@ -83,6 +83,7 @@ _SIGS = {
     "qi21_euler_update": (_I32, [_P, _P, ct.c_double, ct.c_double, _P, ct.c_int64, _P]),
     "qi21_check_device_error": (_I32, [_P, ct.c_size_t, _P]),
     "qi21_status_string": (ct.c_char_p, [_I32]),
+    "qi21_selftest_wait_timeout": (_I32, [_P, ct.c_size_t, ct.c_int64, _P]),
     "qi21_profile_enable": (None, [_I32]),
     "qi21_profile_read": (_I32, [ct.POINTER(qi21_kernel_time), _I32]),
     "qi21_profile_reset": (None, []),
@@ -226,6 +227,10 @@ def qi21_euler_update(x_k, v, sigma_k, sigma_k1, x_out, n, stream=0):
 
 def qi21_check_device_error(ws, ws_bytes, stream=0):
     return lib.qi21_check_device_error(_addr(ws), ws_bytes, stream)
+
+
+def qi21_selftest_wait_timeout(ws, ws_bytes, limit_ns, stream=0):
+    return lib.qi21_selftest_wait_timeout(_addr(ws), ws_bytes, int(limit_ns), stream)
 
 
 def qi21_status_string(s):

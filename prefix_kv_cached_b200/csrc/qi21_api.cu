@@ -717,6 +717,17 @@ extern "C" qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *
     return QI21_OK;
 }
 
+extern "C" qi21_status qi21_selftest_wait_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream) {
+    if (!al16(ws) || ws_bytes < 64) return QI21_ERR_INVALID_ARG;
+    if (limit_ns < 1 || limit_ns > 1000000000) return QI21_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    L.run("selftest_wait_timeout", [&] {
+        sm100::k_selftest_wait_timeout<<<1, 32, 0, st>>>((uint32_t *)ws, (uint64_t)limit_ns);
+    });
+    return finish(L);
+}
+
 extern "C" void qi21_profile_enable(int32_t enable) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof_on = enable != 0;
