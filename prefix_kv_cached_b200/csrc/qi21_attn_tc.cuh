@@ -14,11 +14,12 @@
 //                O  += P_j V_j   (M 128, N Dh, K 128)  -> TMEM O (accumulated across tiles)
 //                P_j (bf16) is read from TMEM, V_j from shared memory as an
 //                MN-major operand.
-//   warps 2..9 : softmax, two threads per query row (TMEM lane): warps w and
-//                w+4 share a lane quadrant and own key columns 0..63 / 64..127
-//                of S_j and the matching half of the O row. The halves swap
-//                their partial row max through shared memory behind a bounded
-//                mbarrier. The row keeps a running max m and only when a tile
+//   warps 2..9 : softmax, two threads per query row: each warp owns 16 TMEM
+//                lanes (16 rows) and reads them with the 16x32bx2 shape, so
+//                threads t and t+16 hold key columns 0..63 / 64..127 of the
+//                same row and the matching halves of its O row; the halves
+//                combine their row max by a shuffle. The row keeps a running
+//                max m and only when a tile
 //                raises it by more than 2^8 (in the exp2 domain) do the two
 //                threads rescale their O halves in TMEM (after PV(j-1) has
 //                landed) — otherwise P_j = exp2(S_j c - m c) <= 256 is formed
@@ -72,8 +73,7 @@ struct AttnCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int OFF_RED = OFF_V + STAGES * KV_BYTES;  // [2][2 halves][128 rows] floats
-    static constexpr int OFF_BAR = OFF_RED + 2 * 2 * BQ * 4;
+    static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
     // The dynamic shared-memory window is checked to start on a 1024-byte
     // boundary (the swizzled tiles need it), so no alignment slack is requested.
     static constexpr size_t SMEM = (size_t)OFF_BAR + 256;
@@ -105,13 +105,10 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t *s_empty = bars + 9;     // [2]
     uint64_t *p_full = bars + 11;     // [2]
     uint64_t *p_empty = bars + 13;    // [2]  (PV of that P buffer done)
-    uint64_t *xchg = bars + 15;       // [2]  (row-max halves exchanged)
-    uint64_t *lx = bars + 17;         //      (row-sum halves exchanged)
-    uint64_t *v_empty = bars + 18;    // [2]  (PV MMA of that V stage done)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+    uint64_t *v_empty = bars + 15;    // [2]  (PV MMA of that V stage done)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *kv_end_s = reinterpret_cast<int *>(tmem_slot + 2);
-    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q0 = blockIdx.x * C::BQ, hh = blockIdx.y, b = blockIdx.z;
@@ -127,9 +124,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(smem_u32(&s_empty[i]), C::SOFTMAX_THREADS);
             mbar_init(smem_u32(&p_full[i]), C::SOFTMAX_THREADS);
             mbar_init(smem_u32(&p_empty[i]), 1);
-            mbar_init(smem_u32(&xchg[i]), C::SOFTMAX_THREADS);
         }
-        mbar_init(smem_u32(lx), C::SOFTMAX_THREADS);
         *abort_flag = 0;
         *kv_end_s = 0;
         fence_barrier_init();
@@ -232,14 +227,18 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else {
         // ---------------------------------------------------------------- softmax warps (2..9)
+        // Warp w owns 16 rows (TMEM lanes 32*(w%4) + 16*((w-2)/4) ..); thread t holds
+        // row t%16, key half t/16 (keys 64h .. 64h+63 of S, O columns h*Dh/2 ..),
+        // loaded with the 16x32bx2 shape, so the two halves of a row meet by shuffle.
         const int quad = warp & 3;
-        const int half = (warp - 2) >> 2;                // key columns half*64 .. +63, O columns half*DH/2 ..
-        const int r = quad * 32 + lane;                  // row within the tile = TMEM lane
+        const int sub = (warp - 2) >> 2;
+        const int rr = lane & 15, half = lane >> 4;
+        const int r = quad * 32 + sub * 16 + rr;          // row within the tile = TMEM lane
         const int row = q0 + r;
         int lim = p.kv_len;
         if (p.kv_limit && row < p.Mq) lim = min(p.kv_limit[row], p.kv_len);
-        const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
-        const uint32_t t_o = t_lane + 256 + half * (DH / 2);
+        const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32 + sub * 16) << 16);
+        const uint32_t t_o = t_lane + 256;
         const float c = p.scale_log2;
         float m_run = -INFINITY, l_half = 0.f;
         bool ok = true;
@@ -256,8 +255,8 @@ __global__ void __launch_bounds__(320, 1)
                 break;
             }
             tc_fence_after();
-            tmem_ld32(t_lane + s * 128 + half * 64, *reinterpret_cast<float(*)[32]>(&sv[0]));
-            tmem_ld32(t_lane + s * 128 + half * 64 + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
+            tmem_ld16x2_32<64>(t_lane + s * 128, *reinterpret_cast<float(*)[32]>(&sv[0]));
+            tmem_ld16x2_32<64>(t_lane + s * 128 + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(smem_u32(&s_empty[s]));
@@ -274,15 +273,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
             float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            // swap the half-row maxima
-            float *red_j = red + (s * 2) * C::BQ;
-            red_j[half * C::BQ + r] = mx;
-            mbar_arrive(smem_u32(&xchg[s]));
-            if (!wait_all(&xchg[s], (j >> 1) & 1)) {
-                ok = false;
-                break;
-            }
-            mx = fmaxf(mx, red_j[(half ^ 1) * C::BQ + r]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));      // the row's other half
             // per row: move the running max only when this tile raises it by more than 2^8
             const bool first = (m_run == -INFINITY);
             const bool grow = first || (mx - m_run) * c > kRescaleLog2;
@@ -299,12 +290,12 @@ __global__ void __launch_bounds__(320, 1)
                 float ov[32];
 #pragma unroll
                 for (int cc = 0; cc < DH / 64; ++cc) {
-                    tmem_ld32(t_o + cc * 32, ov);
+                    tmem_ld16x2_32<DH / 2>(t_o + cc * 32, ov);
                     tmem_wait_ld();
                     uint32_t u[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(ov[i] * alpha);
-                    tmem_st32(t_o + cc * 32, u);
+                    tmem_st16x2_32<DH / 2>(t_o + cc * 32, u);
                 }
                 tmem_wait_st();
             }
@@ -330,25 +321,22 @@ __global__ void __launch_bounds__(320, 1)
                 uint32_t u[32];
 #pragma unroll
                 for (int q = 0; q < 32; ++q) u[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
-                tmem_st32(t_lane + 384 + s * 64 + half * 32, u);
+                tmem_st16x2_32<32>(t_lane + 384 + s * 64, u);
                 tmem_wait_st();
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&p_full[s]));
         }
         if (ok && T > 0) {
-            // combine the half-row sums (the buffer of tile T is free: its readers finished at T-1)
-            float *red_l = red + ((T & 1) * 2) * C::BQ;
-            red_l[half * C::BQ + r] = l_half;
-            mbar_arrive(smem_u32(lx));
-            if (wait_all(lx, 0) && wait_all(&p_empty[(T - 1) & 1], ((T - 1) >> 1) & 1)) {
+            const float l_row = l_half + __shfl_xor_sync(0xffffffffu, l_half, 16);
+            if (wait_all(&p_empty[(T - 1) & 1], ((T - 1) >> 1) & 1)) {
                 tc_fence_after();
-                const float inv = 1.f / (l_half + red_l[(half ^ 1) * C::BQ + r]);
+                const float inv = 1.f / l_row;
                 bf16 *dst = p.out + ((size_t)b * p.Mq + row) * p.d + hh * DH + half * (DH / 2);
                 float ov[32];
 #pragma unroll
                 for (int cc = 0; cc < DH / 64; ++cc) {
-                    tmem_ld32(t_o + cc * 32, ov);          // every lane: the load is warp-collective
+                    tmem_ld16x2_32<DH / 2>(t_o + cc * 32, ov);   // every lane: the load is warp-collective
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) ov[i] *= inv;
