@@ -4,29 +4,36 @@
 // one of the kv_len keys (cached target rows: the target is last, so they see
 // the whole prefix cache and all target keys).
 //
-// One CTA per (item, head, 128 query rows); K and V tiles of 128 keys stream
-// through two 2-stage TMA rings (128-byte swizzle, no multicast).
-//   warp 0     : TMA producers: lane 0 loads Q once, then K_j (a K stage is
-//                released as soon as its S MMA completes); lane 1 loads V_j (a
-//                V stage is released when its PV MMA completes)
+// One CTA per (item, head, 128 query rows). The CTA's T key tiles (128 keys
+// each) are split into two halves, A = tiles [0, TA) and B = tiles [TA, T),
+// TA = ceil(T/2). Each half has its own S and O accumulators in TMEM and its
+// own softmax warpgroup, so the single MMA issuer alternates between them:
+// while half A's softmax turns S_A into P_A, the tensor pipe runs half B's PV
+// and next S, and the other way round. Each half keeps its own running max m
+// and row sum l; the epilogue merges the two partial results,
+//   o = (2^{(m_A-m)c} O_A + 2^{(m_B-m)c} O_B) / (2^{(m_A-m)c} l_A + 2^{(m_B-m)c} l_B),
+// m = max(m_A, m_B) — the standard combination of two softmax partials over
+// disjoint key sets.
+//   warp 0     : TMA producers: lane 0 loads Q once, then the K tiles, lane 1
+//                the V tiles, both in the order A0 B0 A1 B1 ... in which the
+//                MMAs consume them (2-stage rings, 128-byte swizzle, no multicast)
 //   warp 1     : TMEM allocator + UMMA issuer:
-//                S_j = Q K_j^T   (M 128, N 128, K Dh)  -> TMEM S[j % 2]
-//                O  += P_j V_j   (M 128, N Dh, K 128)  -> TMEM O (accumulated across tiles)
-//                P_j (bf16) is read from TMEM, V_j from shared memory as an
-//                MN-major operand.
-//   warps 2..9 : softmax, two threads per query row: each warp owns 16 TMEM
-//                lanes (16 rows) and reads them with the 16x32bx2 shape, so
-//                threads t and t+16 hold key columns 0..63 / 64..127 of the
-//                same row and the matching halves of its O row; the halves
-//                combine their row max by a shuffle. The row keeps a running
-//                max m and only when a tile
-//                raises it by more than 2^8 (in the exp2 domain) do the two
-//                threads rescale their O halves in TMEM (after PV(j-1) has
-//                landed) — otherwise P_j = exp2(S_j c - m c) <= 256 is formed
-//                against the stale max, exactly as the final 1/l normalisation
-//                expects. S_{j+1} and PV(j-1) run under softmax(j).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+Dh), P0 [384,448),
-// P1 [448,512) (P rows as bf16 pairs: key k of row r at lane r, column k/2).
+//                S_X = Q K^T   (M 128, N 128, K Dh)  -> TMEM S_X
+//                O_X += P_X V  (M 128, N Dh, K 128)  -> TMEM O_X, P_X read from
+//                TMEM, V from shared memory as an MN-major operand
+//   warps 2..5 : softmax of half A, one thread per query row (= TMEM lane)
+//   warps 6..9 : softmax of half B
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+Dh), O_B [256+Dh,256+2Dh).
+// P_X (bf16 pairs: key k of row r at lane r, column k/2) overwrites the first 64
+// columns of S_X after the softmax has read all of S_X into registers. The next
+// S_X MMA is issued after the PV MMA that reads P_X; the tcgen05.mma operations
+// of one issuing thread execute in issue order, so that PV reads P_X before the
+// next S_X overwrites it. A commit tracks every earlier MMA of the thread, so
+// when S_X(j) is complete, PV_X(j-1) is too: the softmax may then rescale O_X
+// and write P_X(j) without a further wait.
+// The running max of a row moves only when a tile raises it by more than 2^8
+// (exp2 domain); otherwise P = exp2(S c - m c) <= 256 is formed against the
+// stale max, which the final 1/l normalisation absorbs.
 #pragma once
 #include "qi21_sm100.cuh"
 
@@ -50,6 +57,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for part of the softmax exponentials (the MUFU unit
+// takes the rest): x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f from a
+// cubic with constant term 1 (coefficients: exp2_poly_fit.py, a least-squares
+// relative-error fit, max relative error 1.1e-4 — P is rounded to bf16
+// afterwards, relative step 2^-8); 2^n is added to the exponent field. Inputs
+// below -127 (masked keys: -inf) give exactly +0 (n = -127, f = 0, p = 1).
+__device__ __forceinline__ float ex2_poly(float x) {
+    x = fmaxf(x, -127.f);
+    const float t = x + 12582912.f;            // 1.5 * 2^23: t's low mantissa bits hold rint(x)
+    const float f = x - (t - 12582912.f);
+    float p = fmaf(0.054592825f, f, 0.24221784f);
+    p = fmaf(p, f, 0.6933686f);
+    p = fmaf(p, f, 1.0f);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -63,6 +86,9 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *m, 
         : "memory");
 }
 
+// Named barrier over the 256 softmax threads (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void softmax_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 template <int DH>
 struct AttnCfg {
     static constexpr int BQ = 128, BK = 128;
@@ -74,15 +100,21 @@ struct AttnCfg {
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
     static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+    static constexpr int OFF_STATS = OFF_BAR + 256;        // [2 halves][m, l][128 rows] floats
     // The dynamic shared-memory window is checked to start on a 1024-byte
     // boundary (the swizzled tiles need it), so no alignment slack is requested.
-    static constexpr size_t SMEM = (size_t)OFF_BAR + 256;
+    static constexpr size_t SMEM = (size_t)OFF_STATS + 2 * 2 * BQ * 4;
     static constexpr int THREADS = 320;
-    static constexpr int SOFTMAX_THREADS = 256;
+    static constexpr int HALF_THREADS = 128;               // softmax threads of one half
 };
 
 // Rescale the O row only when the running max grows by more than this (log2 units).
 constexpr float kRescaleLog2 = 8.0f;
+
+// Every POLY-th exponential of a row (POLY > 0) runs on the FMA pipe.
+#ifndef QI21_ATTN_EXP_POLY
+#define QI21_ATTN_EXP_POLY 0
+#endif
 
 template <int DH>
 __global__ void __launch_bounds__(320, 1)
@@ -98,17 +130,17 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t *smem = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;      // [2]
-    uint64_t *v_full = bars + 3;      // [2]
-    uint64_t *k_empty = bars + 5;     // [2]  (S MMA of that K stage done)
-    uint64_t *s_full = bars + 7;      // [2]
-    uint64_t *s_empty = bars + 9;     // [2]
-    uint64_t *p_full = bars + 11;     // [2]
-    uint64_t *p_empty = bars + 13;    // [2]  (PV of that P buffer done)
-    uint64_t *v_empty = bars + 15;    // [2]  (PV MMA of that V stage done)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
+    uint64_t *k_full = bars + 1;      // [2] ring stages
+    uint64_t *k_empty = bars + 3;     // [2] (the S MMA reading that stage is done)
+    uint64_t *v_full = bars + 5;      // [2]
+    uint64_t *v_empty = bars + 7;     // [2] (the PV MMA reading that stage is done)
+    uint64_t *s_full = bars + 9;      // [2 halves]
+    uint64_t *p_full = bars + 11;     // [2 halves] (softmax wrote P and finished with O)
+    uint64_t *o_full = bars + 13;     // every MMA done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *kv_end_s = reinterpret_cast<int *>(tmem_slot + 2);
+    float *stats = reinterpret_cast<float *>(smem + C::OFF_STATS);   // [half][m | l][row]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q0 = blockIdx.x * C::BQ, hh = blockIdx.y, b = blockIdx.z;
@@ -117,14 +149,13 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(smem_u32(q_full), 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&k_full[i]), 1);
-            mbar_init(smem_u32(&v_full[i]), 1);
             mbar_init(smem_u32(&k_empty[i]), 1);
+            mbar_init(smem_u32(&v_full[i]), 1);
             mbar_init(smem_u32(&v_empty[i]), 1);
             mbar_init(smem_u32(&s_full[i]), 1);
-            mbar_init(smem_u32(&s_empty[i]), C::SOFTMAX_THREADS);
-            mbar_init(smem_u32(&p_full[i]), C::SOFTMAX_THREADS);
-            mbar_init(smem_u32(&p_empty[i]), 1);
+            mbar_init(smem_u32(&p_full[i]), C::HALF_THREADS);
         }
+        mbar_init(smem_u32(o_full), 1);
         *abort_flag = 0;
         *kv_end_s = 0;
         fence_barrier_init();
@@ -147,68 +178,51 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tmem_base = *tmem_slot;
     const int kv_end = *kv_end_s;
     const int T = (kv_end + C::BK - 1) / C::BK;
+    const int TA = (T + 1) >> 1, TB = T >> 1;     // tiles of half A and half B
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producers
-        // lane 0 streams K (a stage frees as soon as its S MMA is done, so K runs
-        // two tiles ahead); lane 1 streams V (a stage frees after its PV MMA).
+        // Load n of either ring is key tile A(n/2) for even n, B(n/2) for odd n.
         if (lane == 0 && T > 0) {
             const uint32_t qb = smem_u32(q_full);
             mbar_arrive_expect_tx(qb, C::Q_BYTES);
             for (int x = 0; x < C::BOXES; ++x)
                 tma_load_4d(smem_u32(smem + C::OFF_Q + x * (C::BQ * 128)), &tmQ, qb, hh * DH + x * 64,
                             b * p.Mq + q0, 0, 0);
-            for (int j = 0; j < T; ++j) {
-                const int s = j & 1;
-                if (!mbar_wait(smem_u32(&k_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+            for (int n = 0; n < T; ++n) {
+                const int s = n & 1, tile = (n & 1) ? TA + (n >> 1) : (n >> 1);
+                if (!mbar_wait(smem_u32(&k_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, p.err)) break;
                 const uint32_t kb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(kb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
                     tma_load_4d(smem_u32(smem + C::OFF_K + s * C::KV_BYTES + x * (C::BK * 128)), &tmK, kb,
-                                hh * DH + x * 64, j * C::BK, b, p.layer);
+                                hh * DH + x * 64, tile * C::BK, b, p.layer);
             }
         } else if (lane == 1 && T > 0) {
-            for (int j = 0; j < T; ++j) {
-                const int s = j & 1;
-                if (!mbar_wait(smem_u32(&v_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+            for (int n = 0; n < T; ++n) {
+                const int s = n & 1, tile = (n & 1) ? TA + (n >> 1) : (n >> 1);
+                if (!mbar_wait(smem_u32(&v_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, p.err)) break;
                 const uint32_t vb = smem_u32(&v_full[s]);
                 mbar_arrive_expect_tx(vb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
                     tma_load_4d(smem_u32(smem + C::OFF_V + s * C::KV_BYTES + x * (C::BK * 128)), &tmV, vb,
-                                hh * DH + x * 64, j * C::BK, b, p.layer);
+                                hh * DH + x * 64, tile * C::BK, b, p.layer);
             }
         }
     } else if (warp == 1) {
         if (lane == 0 && T > 0) {
             // ------------------------------------------------------------ UMMA issuer
+            // order: S_A0 S_B0 | PV_A0 S_A1 PV_B0 S_B1 | PV_A1 S_A2 PV_B1 S_B2 | ...
             constexpr uint32_t idesc_s = idesc_bf16_f32(C::BQ, C::BK);
             constexpr uint32_t idesc_o = idesc_bf16_f32(C::BQ, DH, true);
             const uint32_t sq = smem_u32(smem + C::OFF_Q);
-            const uint32_t o_tmem = tmem_base + 256;
-            bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.err);
-            auto issue_pv = [&](int i) -> bool {
-                const int s = i & 1;
-                if (!mbar_wait(smem_u32(&p_full[s]), (i >> 1) & 1, abort_flag, p.err)) return false;
-                if (!mbar_wait(smem_u32(&v_full[s]), (i >> 1) & 1, abort_flag, p.err)) return false;
-                tc_fence_after();
-                const uint32_t p_tmem = tmem_base + 384 + s * 64;
-                const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
-#pragma unroll
-                for (int k = 0; k < C::BK / 16; ++k) {
-                    const uint64_t bdesc = sdesc_mnmajor_sw128(sv + k * 2048, C::BK * 128);
-                    umma_f16_ts(o_tmem, p_tmem + k * 8, bdesc, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
-                }
-                umma_commit(smem_u32(&p_empty[s]));
-                umma_commit(smem_u32(&v_empty[s]));
-                return true;
-            };
-            for (int j = 0; j < T && ok; ++j) {
-                const int s = j & 1;
-                if (!mbar_wait(smem_u32(&k_full[s]), (j >> 1) & 1, abort_flag, p.err)) break;
-                if (!mbar_wait(smem_u32(&s_empty[s]), ((j >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+            int nk = 0, nv = 0;                      // loads consumed from the K and V rings
+            auto issue_s = [&](int h) -> bool {
+                const int s = nk & 1;
+                if (!mbar_wait(smem_u32(&k_full[s]), (nk >> 1) & 1, abort_flag, p.err)) return false;
                 tc_fence_after();
                 const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KV_BYTES);
-                const uint32_t d_tmem = tmem_base + s * 128;
+                const uint32_t d_tmem = tmem_base + h * 128;
 #pragma unroll
                 for (int k = 0; k < DH / 16; ++k) {
                     const uint32_t off = (k >> 2) * (C::BQ * 128) + (k & 3) * 32;
@@ -216,132 +230,170 @@ __global__ void __launch_bounds__(320, 1)
                              sdesc_kmajor_sw128(sk + (k >> 2) * (C::BK * 128) + (k & 3) * 32), idesc_s,
                              k > 0 ? 1u : 0u);
                 }
-                umma_commit(smem_u32(&s_full[s]));
+                umma_commit(smem_u32(&s_full[h]));
                 umma_commit(smem_u32(&k_empty[s]));
-                if (j >= 1 && !issue_pv(j - 1)) {
-                    ok = false;
-                    break;
+                ++nk;
+                return true;
+            };
+            auto issue_pv = [&](int h, int j) -> bool {
+                if (!mbar_wait(smem_u32(&p_full[h]), j & 1, abort_flag, p.err)) return false;
+                const int s = nv & 1;
+                if (!mbar_wait(smem_u32(&v_full[s]), (nv >> 1) & 1, abort_flag, p.err)) return false;
+                tc_fence_after();
+                const uint32_t p_tmem = tmem_base + h * 128;
+                const uint32_t o_tmem = tmem_base + 256 + h * DH;
+                const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
+#pragma unroll
+                for (int k = 0; k < C::BK / 16; ++k) {
+                    const uint64_t bdesc = sdesc_mnmajor_sw128(sv + k * 2048, C::BK * 128);
+                    umma_f16_ts(o_tmem, p_tmem + k * 8, bdesc, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&v_empty[s]));
+                ++nv;
+                return true;
+            };
+            bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.err);
+            ok = ok && issue_s(0);
+            if (TB > 0) ok = ok && issue_s(1);
+            for (int j = 0; j < TA && ok; ++j) {
+                ok = issue_pv(0, j);
+                if (ok && j + 1 < TA) ok = issue_s(0);
+                if (ok && j < TB) {
+                    ok = issue_pv(1, j);
+                    if (ok && j + 1 < TB) ok = issue_s(1);
                 }
             }
-            if (ok) issue_pv(T - 1);
+            if (ok) umma_commit(smem_u32(o_full));
         }
     } else {
         // ---------------------------------------------------------------- softmax warps (2..9)
-        // Warp w owns 16 rows (TMEM lanes 32*(w%4) + 16*((w-2)/4) ..); thread t holds
-        // row t%16, key half t/16 (keys 64h .. 64h+63 of S, O columns h*Dh/2 ..),
-        // loaded with the 16x32bx2 shape, so the two halves of a row meet by shuffle.
-        const int quad = warp & 3;
-        const int sub = (warp - 2) >> 2;
-        const int rr = lane & 15, half = lane >> 4;
-        const int r = quad * 32 + sub * 16 + rr;          // row within the tile = TMEM lane
+        const int h = (warp - 2) >> 2;                 // half: 0 = A (warps 2..5), 1 = B (warps 6..9)
+        const int quad = warp & 3;                     // the TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;                // row within the tile = TMEM lane
         const int row = q0 + r;
         int lim = p.kv_len;
         if (p.kv_limit && row < p.Mq) lim = min(p.kv_limit[row], p.kv_len);
-        const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32 + sub * 16) << 16);
-        const uint32_t t_o = t_lane + 256;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
+        const uint32_t t_s = t_lane + h * 128;         // S_h, later P_h in its first 64 columns
+        const uint32_t t_o = t_lane + 256 + h * DH;    // O_h
+        const int nt = h ? TB : TA, tile0 = h ? TA : 0;
         const float c = p.scale_log2;
-        float m_run = -INFINITY, l_half = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        float sv[64];
         // tcgen05.ld / tcgen05.st are warp-collective (.sync.aligned): every
         // decision that guards one is made uniform across the warp.
         auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag, p.err) ? 1 : 0) != 0;
         };
-        for (int j = 0; j < T && ok; ++j) {
-            const int s = j & 1;
-            if (!wait_all(&s_full[s], (j >> 1) & 1)) {
+        for (int j = 0; j < nt && ok; ++j) {
+            if (!wait_all(&s_full[h], j & 1)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            tmem_ld16x2_32<64>(t_lane + s * 128, *reinterpret_cast<float(*)[32]>(&sv[0]));
-            tmem_ld16x2_32<64>(t_lane + s * 128 + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(smem_u32(&s_empty[s]));
-            const int key0 = j * C::BK + half * 64;
-            if (key0 + 64 > lim) {
+            float sv[4][32];                          // S row: key 32a+b in sv[a][b]
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (key0 + i >= lim) sv[i] = -INFINITY;
+            for (int cc = 0; cc < 4; ++cc) tmem_ld32(t_s + cc * 32, sv[cc]);
+            tmem_wait_ld();
+            const int key0 = (tile0 + j) * C::BK;
+            if (key0 + C::BK > lim) {
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                    if (key0 + i >= lim) sv[i >> 5][i & 31] = -INFINITY;
             }
             float m8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = sv[i];
+            for (int i = 0; i < 8; ++i) m8[i] = sv[0][i];
 #pragma unroll
-            for (int i = 8; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
-            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));      // the row's other half
-            // per row: move the running max only when this tile raises it by more than 2^8
+            for (int i = 8; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i >> 5][i & 31]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            // move the running max only when this tile raises it by more than 2^8
             const bool first = (m_run == -INFINITY);
             const bool grow = first || (mx - m_run) * c > kRescaleLog2;
             const float m_new = grow ? fmaxf(m_run, mx) : m_run;
             const float alpha = (grow && !first) ? ex2_approx((m_run - m_new) * c) : 1.f;
-            if (__any_sync(0xffffffffu, grow && !first)) {
-                // O holds PV(0..j-1) against the old max: the whole warp rescales its
-                // O rows (alpha = 1 where the row's max did not move) once PV(j-1) landed
-                if (!wait_all(&p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                float ov[32];
-#pragma unroll
-                for (int cc = 0; cc < DH / 64; ++cc) {
-                    tmem_ld16x2_32<DH / 2>(t_o + cc * 32, ov);
-                    tmem_wait_ld();
-                    uint32_t u[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(ov[i] * alpha);
-                    tmem_st16x2_32<DH / 2>(t_o + cc * 32, u);
-                }
-                tmem_wait_st();
-            }
-            l_half *= alpha;
+            l_run *= alpha;
             m_run = m_new;
-            const float mc = m_run * c;
+            // a row with no allowed key so far (half B past its limit) keeps m = -inf: P = 0
+            const float mc = m_run == -INFINITY ? 0.f : m_run * c;
             float s8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) s8[i] = 0.f;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                sv[i] = ex2_approx(fmaf(sv[i], c, -mc));    // masked: exp2(-inf) = 0
-                s8[i & 7] += sv[i];
-            }
-            l_half += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-            // P buffer s is free once PV(j-2) has completed
-            if (!wait_all(&p_empty[s], ((j >> 1) & 1) ^ 1)) {
-                ok = false;
-                break;
-            }
-            // this half's 64 keys -> 32 TMEM columns of P[s] (bf16 pairs, lower key in the low half)
-            {
-                uint32_t u[32];
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t u[16];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) u[q] = pack_bf16x2(sv[2 * q], sv[2 * q + 1]);
-                tmem_st16x2_32<32>(t_lane + 384 + s * 64, u);
-                tmem_wait_st();
+                for (int q = 0; q < 16; ++q) {
+                    float e[2];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const float x = fmaf(sv[cc][2 * q + t], c, -mc);   // masked: -inf -> 0
+#if QI21_ATTN_EXP_POLY > 0
+                        e[t] = ((2 * q + t) % QI21_ATTN_EXP_POLY == QI21_ATTN_EXP_POLY - 1) ? ex2_poly(x)
+                                                                                          : ex2_approx(x);
+#else
+                        e[t] = ex2_approx(x);
+#endif
+                    }
+                    s8[(2 * q) & 7] += e[0];
+                    s8[(2 * q + 1) & 7] += e[1];
+                    u[q] = pack_bf16x2(e[0], e[1]);
+                }
+                tmem_st16(t_s + cc * 16, u);               // P_h: keys 32cc .. 32cc+31
             }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&p_full[s]));
-        }
-        if (ok && T > 0) {
-            const float l_row = l_half + __shfl_xor_sync(0xffffffffu, l_half, 16);
-            if (wait_all(&p_empty[(T - 1) & 1], ((T - 1) >> 1) & 1)) {
-                tc_fence_after();
-                const float inv = 1.f / l_row;
-                bf16 *dst = p.out + ((size_t)b * p.Mq + row) * p.d + hh * DH + half * (DH / 2);
+            if (__any_sync(0xffffffffu, grow && !first)) {
+                // O_h holds PV_h(0..j-1) against the old max (complete: S_h(j) was
+                // issued after PV_h(j-1)); alpha = 1 on rows whose max did not move.
+                // Done after P so that the S registers are free.
                 float ov[32];
 #pragma unroll
-                for (int cc = 0; cc < DH / 64; ++cc) {
-                    tmem_ld16x2_32<DH / 2>(t_o + cc * 32, ov);   // every lane: the load is warp-collective
+                for (int cc = 0; cc < DH / 32; ++cc) {
+                    tmem_ld32(t_o + cc * 32, ov);
                     tmem_wait_ld();
+                    uint32_t u[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] *= inv;
-                    if (row < p.Mq) store_bf16x32(dst + cc * 32, ov);
+                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(ov[i] * alpha);
+                    tmem_st32(t_o + cc * 32, u);
                 }
+                tmem_wait_st();
+            }
+            tmem_wait_st();
+            l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+            tc_fence_before();
+            mbar_arrive(smem_u32(&p_full[h]));
+        }
+        // merge the halves: each publishes its (m, l) per row; half h then writes
+        // output columns [h Dh/2, (h+1) Dh/2) of its rows from O_A and O_B
+        stats[(2 * h + 0) * C::BQ + r] = m_run;
+        stats[(2 * h + 1) * C::BQ + r] = l_run;
+        softmax_bar_sync();
+        if (ok && T > 0 && wait_all(o_full, 0)) {
+            tc_fence_after();
+            const float mA = stats[0 * C::BQ + r], lA = stats[1 * C::BQ + r];
+            const float mB = stats[2 * C::BQ + r], lB = stats[3 * C::BQ + r];
+            float m = fmaxf(mA, mB);
+            if (m == -INFINITY) m = 0.f;
+            const float wA = ex2_approx((mA - m) * c);
+            const float wB = TB > 0 ? ex2_approx((mB - m) * c) : 0.f;
+            const float inv = 1.f / (lA * wA + lB * wB);
+            const float fA = wA * inv, fB = wB * inv;
+            bf16 *dst = p.out + ((size_t)b * p.Mq + row) * p.d + hh * DH + h * (DH / 2);
+#pragma unroll
+            for (int cc = 0; cc < DH / 64; ++cc) {
+                const int col = h * (DH / 2) + cc * 32;
+                float oa[32], ob[32];
+                tmem_ld32(t_lane + 256 + col, oa);            // every lane: the loads are warp-collective
+                if (TB > 0) tmem_ld32(t_lane + 256 + DH + col, ob);
+                tmem_wait_ld();
+                if (TB > 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) oa[i] = fmaf(fA, oa[i], fB * ob[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) oa[i] *= fA;
+                }
+                if (row < p.Mq) store_bf16x32(dst + cc * 32, oa);
             }
         }
     }

@@ -85,6 +85,8 @@ WORKLOADS: Dict[str, Workload] = {
     # Test-only: several 128-row tiles with ragged tails, two batch items.
     "small": Workload("small", SMALL, 2, (_text(77), _img(11, 11), _img(15, 20)), TURBO_SIGMAS, 1234),
     "small64": Workload("small64", SMALL64, 2, (_text(40), _img(9, 10), _img(10, 13)), TURBO_SIGMAS, 1234),
+    # Test-only: every attention pass fits one 128-key tile (P 56, N 64).
+    "small_t1": Workload("small_t1", SMALL, 1, (_text(20), _img(6, 6), _img(8, 8)), TURBO_SIGMAS, 1234),
     # Single full-width block.
     "block": Workload("block", BLOCK, 1, (_text(512), _img(64, 64), _img(64, 64)), TURBO_SIGMAS, 1234),
     "mid": Workload("mid", MID, 8, (_text(256), _img(16, 16), _img(16, 16)), TURBO_SIGMAS, 1234),

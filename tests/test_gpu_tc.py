@@ -64,7 +64,7 @@ def test_tc_family_agrees_with_cuda_core_family(B, name):
     assert rel_l2(a[3], b[3]) < 1e-2           # full recompute
 
 
-@pytest.mark.parametrize("name", ["small", "small64"])
+@pytest.mark.parametrize("name", ["small", "small64", "small_t1"])
 def test_tc_matches_oracle(B, name):
     w = C.make_workload(name)
     model, wts = oracle_model(w, "bfloat16")
