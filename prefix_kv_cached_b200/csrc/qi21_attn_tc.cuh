@@ -17,7 +17,7 @@
 //   warp 0     : TMA producers: lane 0 loads Q once, then the K tiles, lane 1
 //                the V tiles, both in the order A0 B0 A1 B1 ... in which the
 //                MMAs consume them (2-stage rings, 128-byte swizzle, no multicast)
-//   warp 1     : TMEM allocator + UMMA issuer:
+//   warp 1     : TMEM allocator + UMMA issuer (warp-uniform schedule, one elected lane issues):
 //                S_X = Q K^T   (M 128, N 128, K Dh)  -> TMEM S_X
 //                O_X += P_X V  (M 128, N Dh, K 128)  -> TMEM O_X, P_X read from
 //                TMEM, V from shared memory as an MN-major operand
@@ -95,16 +95,16 @@ struct AttnCfg {
     static constexpr int BOXES = DH / 64;                  // 64-element (128-byte) swizzle boxes per row
     static constexpr int Q_BYTES = BQ * DH * 2;
     static constexpr int KV_BYTES = BK * DH * 2;           // one K or V tile
-    static constexpr int STAGES = 2;
+    static constexpr int SK = 2, SV = 2;                   // K and V ring stages
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
-    static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+    static constexpr int OFF_V = OFF_K + SK * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + SV * KV_BYTES;
     static constexpr int OFF_STATS = OFF_BAR + 256;        // [2 halves][m, l][128 rows] floats
     // The dynamic shared-memory window is checked to start on a 1024-byte
     // boundary (the swizzled tiles need it), so no alignment slack is requested.
     static constexpr size_t SMEM = (size_t)OFF_STATS + 2 * 2 * BQ * 4;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 320;                    // warps: 0 loads, 1 MMA, 2..9 softmax
     static constexpr int HALF_THREADS = 128;               // softmax threads of one half
 };
 
@@ -130,14 +130,15 @@ __global__ void __launch_bounds__(320, 1)
     uint8_t *smem = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;      // [2] ring stages
-    uint64_t *k_empty = bars + 3;     // [2] (the S MMA reading that stage is done)
-    uint64_t *v_full = bars + 5;      // [2]
-    uint64_t *v_empty = bars + 7;     // [2] (the PV MMA reading that stage is done)
-    uint64_t *s_full = bars + 9;      // [2 halves]
-    uint64_t *p_full = bars + 11;     // [2 halves] (softmax wrote P and finished with O)
-    uint64_t *o_full = bars + 13;     // every MMA done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+    uint64_t *k_full = q_full + 1;     // [SK] ring stages
+    uint64_t *k_empty = k_full + C::SK;   // [SK] (the S MMA reading that stage is done)
+    uint64_t *v_full = k_empty + C::SK;   // [SV]
+    uint64_t *v_empty = v_full + C::SV;   // [SV] (the PV MMA reading that stage is done)
+    uint64_t *s_full = v_empty + C::SV;   // [2 halves]
+    uint64_t *p_full = s_full + 2;        // [2 halves] (softmax wrote P and finished with O)
+    uint64_t *o_full = p_full + 2;        // every MMA done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
+    static_assert((1 + 2 * C::SK + 2 * C::SV + 5) * 8 + 16 <= 256, "barrier region");
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *kv_end_s = reinterpret_cast<int *>(tmem_slot + 2);
     float *stats = reinterpret_cast<float *>(smem + C::OFF_STATS);   // [half][m | l][row]
@@ -147,11 +148,15 @@ __global__ void __launch_bounds__(320, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(q_full), 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::SK; ++i) {
             mbar_init(smem_u32(&k_full[i]), 1);
             mbar_init(smem_u32(&k_empty[i]), 1);
+        }
+        for (int i = 0; i < C::SV; ++i) {
             mbar_init(smem_u32(&v_full[i]), 1);
             mbar_init(smem_u32(&v_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
             mbar_init(smem_u32(&p_full[i]), C::HALF_THREADS);
         }
@@ -190,8 +195,8 @@ __global__ void __launch_bounds__(320, 1)
                 tma_load_4d(smem_u32(smem + C::OFF_Q + x * (C::BQ * 128)), &tmQ, qb, hh * DH + x * 64,
                             b * p.Mq + q0, 0, 0);
             for (int n = 0; n < T; ++n) {
-                const int s = n & 1, tile = (n & 1) ? TA + (n >> 1) : (n >> 1);
-                if (!mbar_wait(smem_u32(&k_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+                const int s = n % C::SK, tile = (n & 1) ? TA + (n >> 1) : (n >> 1);
+                if (!mbar_wait(smem_u32(&k_empty[s]), ((n / C::SK) & 1) ^ 1, abort_flag, p.err)) break;
                 const uint32_t kb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(kb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
@@ -200,8 +205,8 @@ __global__ void __launch_bounds__(320, 1)
             }
         } else if (lane == 1 && T > 0) {
             for (int n = 0; n < T; ++n) {
-                const int s = n & 1, tile = (n & 1) ? TA + (n >> 1) : (n >> 1);
-                if (!mbar_wait(smem_u32(&v_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, p.err)) break;
+                const int s = n % C::SV, tile = (n & 1) ? TA + (n >> 1) : (n >> 1);
+                if (!mbar_wait(smem_u32(&v_empty[s]), ((n / C::SV) & 1) ^ 1, abort_flag, p.err)) break;
                 const uint32_t vb = smem_u32(&v_full[s]);
                 mbar_arrive_expect_tx(vb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
@@ -210,49 +215,61 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && T > 0) {
+        if (T > 0) {
             // ------------------------------------------------------------ UMMA issuer
             // order: S_A0 S_B0 | PV_A0 S_A1 PV_B0 S_B1 | PV_A1 S_A2 PV_B1 S_B2 | ...
+            // The whole warp runs the schedule (its values stay warp-uniform) and one
+            // elected lane issues each group of MMAs. Descriptors are built once; a
+            // K=16 step inside a 64-element swizzle box adds 32 B (2 units of the
+            // start-address field), a new box adds rows * 128 B, a new V K-step 2 KB.
             constexpr uint32_t idesc_s = idesc_bf16_f32(C::BQ, C::BK);
             constexpr uint32_t idesc_o = idesc_bf16_f32(C::BQ, DH, true);
-            const uint32_t sq = smem_u32(smem + C::OFF_Q);
+            constexpr uint32_t BOX_UNITS = (C::BK * 128) >> 4;     // Q (BQ == BK) and K boxes
+            constexpr uint32_t KV_UNITS = C::KV_BYTES >> 4;
+            const uint64_t dq0 = sdesc_kmajor_sw128(smem_u32(smem + C::OFF_Q));
+            const uint64_t dk0 = sdesc_kmajor_sw128(smem_u32(smem + C::OFF_K));
+            const uint64_t dv0 = sdesc_mnmajor_sw128(smem_u32(smem + C::OFF_V), C::BK * 128);
+            const bool leader = elect_one();
+            auto wait_warp = [&](uint64_t *bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag, p.err) ? 1 : 0) != 0;
+            };
             int nk = 0, nv = 0;                      // loads consumed from the K and V rings
             auto issue_s = [&](int h) -> bool {
-                const int s = nk & 1;
-                if (!mbar_wait(smem_u32(&k_full[s]), (nk >> 1) & 1, abort_flag, p.err)) return false;
+                const int s = nk % C::SK;
+                if (!wait_warp(&k_full[s], (nk / C::SK) & 1)) return false;
                 tc_fence_after();
-                const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KV_BYTES);
-                const uint32_t d_tmem = tmem_base + h * 128;
+                if (leader) {
+                    const uint64_t dk = dk0 + s * KV_UNITS;
 #pragma unroll
-                for (int k = 0; k < DH / 16; ++k) {
-                    const uint32_t off = (k >> 2) * (C::BQ * 128) + (k & 3) * 32;
-                    umma_f16(d_tmem, sdesc_kmajor_sw128(sq + off),
-                             sdesc_kmajor_sw128(sk + (k >> 2) * (C::BK * 128) + (k & 3) * 32), idesc_s,
-                             k > 0 ? 1u : 0u);
+                    for (int k = 0; k < DH / 16; ++k) {
+                        const uint32_t off = (k >> 2) * BOX_UNITS + (k & 3) * 2;
+                        umma_f16(tmem_base + h * 128, dq0 + off, dk + off, idesc_s, k > 0 ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&s_full[h]));
+                    umma_commit(smem_u32(&k_empty[s]));
                 }
-                umma_commit(smem_u32(&s_full[h]));
-                umma_commit(smem_u32(&k_empty[s]));
+                __syncwarp();
                 ++nk;
                 return true;
             };
             auto issue_pv = [&](int h, int j) -> bool {
-                if (!mbar_wait(smem_u32(&p_full[h]), j & 1, abort_flag, p.err)) return false;
-                const int s = nv & 1;
-                if (!mbar_wait(smem_u32(&v_full[s]), (nv >> 1) & 1, abort_flag, p.err)) return false;
+                if (!wait_warp(&p_full[h], j & 1)) return false;
+                const int s = nv % C::SV;
+                if (!wait_warp(&v_full[s], (nv / C::SV) & 1)) return false;
                 tc_fence_after();
-                const uint32_t p_tmem = tmem_base + h * 128;
-                const uint32_t o_tmem = tmem_base + 256 + h * DH;
-                const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
+                if (leader) {
+                    const uint64_t dv = dv0 + s * KV_UNITS;
 #pragma unroll
-                for (int k = 0; k < C::BK / 16; ++k) {
-                    const uint64_t bdesc = sdesc_mnmajor_sw128(sv + k * 2048, C::BK * 128);
-                    umma_f16_ts(o_tmem, p_tmem + k * 8, bdesc, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < C::BK / 16; ++k)
+                        umma_f16_ts(tmem_base + 256 + h * DH, tmem_base + h * 128 + k * 8, dv + k * 128, idesc_o,
+                                    (j > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(smem_u32(&v_empty[s]));
                 }
-                umma_commit(smem_u32(&v_empty[s]));
+                __syncwarp();
                 ++nv;
                 return true;
             };
-            bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.err);
+            bool ok = wait_warp(q_full, 0);
             ok = ok && issue_s(0);
             if (TB > 0) ok = ok && issue_s(1);
             for (int j = 0; j < TA && ok; ++j) {
@@ -263,7 +280,8 @@ __global__ void __launch_bounds__(320, 1)
                     if (ok && j + 1 < TB) ok = issue_s(1);
                 }
             }
-            if (ok) umma_commit(smem_u32(o_full));
+            if (ok && leader) umma_commit(smem_u32(o_full));
+            __syncwarp();
         }
     } else {
         // ---------------------------------------------------------------- softmax warps (2..9)

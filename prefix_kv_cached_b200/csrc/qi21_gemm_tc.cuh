@@ -197,41 +197,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- UMMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN);
-            int stage = 0;
-            uint32_t phase = 0;
-            int it = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-                int m_blk, n_blk, kb0, kb1;
-                tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
-                const int acc = it & 1;
-                const uint32_t acc_phase = (it >> 1) & 1;
-                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, p.err)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, p.err)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(stage_base + (size_t)stage * TC_STAGE_BYTES);
-                    const uint32_t sb = sa + TC_A_BYTES;
-#pragma unroll
-                    for (int k = 0; k < TC_BK / 16; ++k) {
-                        umma_f16(d_tmem, sdesc_kmajor_sw128(sa + k * 32), sdesc_kmajor_sw128(sb + k * 32), idesc,
-                                 (kb > kb0 || k > 0) ? 1u : 0u);
-                    }
-                    umma_commit(smem_u32(&empty[stage]));
-                    if (++stage == TC_STAGES) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
+        // The whole warp runs the schedule and one elected lane issues; the
+        // operand descriptors are built once and advanced by adding to the
+        // start-address field (16-byte units: 32 B per K=16 step).
+        constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN);
+        constexpr uint32_t STAGE_UNITS = TC_STAGE_BYTES >> 4, A_UNITS = TC_A_BYTES >> 4;
+        const uint64_t d0 = sdesc_kmajor_sw128(smem_u32(stage_base));
+        const bool leader = elect_one();
+        auto wait_warp = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag, p.err) ? 1 : 0) != 0;
+        };
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+            int m_blk, n_blk, kb0, kb1;
+            tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!wait_warp(&tempty[acc], acc_phase ^ 1)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!wait_warp(&full[stage], phase)) {
+                    ok = false;
+                    break;
                 }
-                if (ok) umma_commit(smem_u32(&tfull[acc]));
+                tc_fence_after();
+                if (leader) {
+                    const uint64_t da = d0 + (uint32_t)stage * STAGE_UNITS;
+#pragma unroll
+                    for (int k = 0; k < TC_BK / 16; ++k)
+                        umma_f16(d_tmem, da + 2 * k, da + A_UNITS + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                    umma_commit(smem_u32(&empty[stage]));
+                }
+                __syncwarp();
+                if (++stage == TC_STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
             }
+            if (ok && leader) umma_commit(smem_u32(&tfull[acc]));
+            __syncwarp();
         }
     } else {
         // ---------------------------------------------------------- epilogue (warps 2..5)
