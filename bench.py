@@ -167,7 +167,14 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
-def oracle_sample(w, rows=512, seed=4321):
+# Target rows of the one-block oracle sample behind `cpu_baseline` (about 10-30 s of
+# host work at full width); the reference arm times 512-row samples per step so that
+# its warm-up + timed steps end within a few minutes.
+CPU_BASELINE_ROWS = 4096
+REFERENCE_ROWS = 512
+
+
+def oracle_sample(w, rows=REFERENCE_ROWS, seed=4321):
     """Time the fp64 oracle on a bounded sample of the workload: one block of
     the cached step at full width for `rows` target tokens attending to all
     P + N keys (the other targets' K/V are synthetic cache rows). Returns
@@ -264,7 +271,7 @@ def run_reference(args, w, world, rank):
         if i >= args.warmup:
             steps.append(dt)
     dt = statistics.mean(steps)
-    rows = min(512, w.n_target)
+    rows = min(REFERENCE_ROWS, w.n_target)
     tok_s = rows / (dt * w.shape.n_layers)
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
@@ -441,7 +448,7 @@ def main():
             "roofline": roof, "kernels": kernels, "gpu_launches": launches[0], "clocks": clk, "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
-            dt, tok_s, threads, desc = oracle_sample(w)
+            dt, tok_s, threads, desc = oracle_sample(w, rows=CPU_BASELINE_ROWS)
             line["cpu_baseline"] = {"value": round(tok_s, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
                                     "sample": desc, "seconds": round(dt, 2)}
         print(json.dumps(line), flush=True)
