@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the whole-image CUDA-graph timing")
     return ap.parse_args()
 
 
@@ -366,8 +367,11 @@ def main():
     clocks.start()
     time.sleep(0.3)
     t0.record(st)
+    marks = []
     for k in range(args.steps):
         step(k)
+        marks.append(torch.cuda.Event(enable_timing=True))
+        marks[-1].record(st)
     t1.record(st)
     torch.cuda.synchronize()
     dist_barrier(world)
@@ -379,6 +383,35 @@ def main():
     ms_max, value = aggregate(world, tokens, args.steps, ms)
     r.check_device()
     ms_step = ms_max / args.steps
+    per_step = [t0.elapsed_time(marks[0])] + [marks[i - 1].elapsed_time(marks[i]) for i in range(1, len(marks))]
+    pct = {f"p{q}": round(float(np.percentile(per_step, q)), 3) for q in (50, 95, 99)}
+
+    # the whole image (extract + every cached step + Euler) as one CUDA graph whose
+    # sigma schedule is read from a device table
+    image = None
+    if not args.no_graph:
+        sig_dev = torch.tensor([float(s_) for s_ in sig], dtype=torch.float64, device=dev)
+        xg = x0.clone()
+        graph = r.capture_image(pre, xg, sig_dev)
+        xg.copy_(x0)
+        graph.replay()
+        torch.cuda.synchronize()
+        r.check_device()
+        reps = 3
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist_barrier(world)
+        torch.cuda.synchronize()
+        g0.record(st)
+        for _ in range(reps):
+            xg.copy_(x0)
+            graph.replay()
+        g1.record(st)
+        torch.cuda.synchronize()
+        img_ms = dist_max(g0.elapsed_time(g1), world) / reps
+        image = {"image_ms": round(img_ms, 3), "tokens_per_s": round(world * tokens / (img_ms / 1e3), 1),
+                 "steps": len(sig) - 1, "how": "one CUDA graph per image: t=0 modulation, prefix extract, "
+                 "then per step modulation from the device sigma table, cached step, Euler"}
+        del graph
 
     # e2e: same step through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -443,8 +476,10 @@ def main():
             "config": config_dict(w),
             "tensor_frac_step": round(step_tflops / peaks["bf16_tflops_sustained"], 4),
             "step_tflops": round(step_tflops, 1),
+            "step_ms_percentiles": pct,
             "per_image": {"extract_ms": round(extract_ms, 3),
-                          "tokens_per_s": round(world * tokens / ((extract_ms + 8 * ms_step) / 1e3), 1)},
+                          "tokens_per_s": round(world * tokens / ((extract_ms + 8 * ms_step) / 1e3), 1),
+                          "graph": image},
             "roofline": roof, "kernels": kernels, "gpu_launches": launches[0], "clocks": clk, "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -249,6 +249,43 @@ qi21_status qi21_full_recompute_step(const qi21_config *cfg, const qi21_weights 
 qi21_status qi21_euler_update(const float *x_k, const float *v, double sigma_k, double sigma_k1,
                               float *x_out, int64_t n, void *stream);
 
+/* Device-indexed forms for captured sequences (CUDA graphs): the sigma of a
+ * step is read on the device from sigmas, a table of float64 values in device
+ * memory (8-byte aligned, caller-owned, at least step + 2 entries), so one
+ * captured sequence serves any sigma schedule written into the table before a
+ * replay. qi21_modulation_at computes the embedding of t = t_per_sigma *
+ * sigmas[step] on the device in fp64 (the pages use t = 1000 * sigma, [3B] §1;
+ * [6B] §3) and otherwise equals qi21_modulation; qi21_euler_update_at applies
+ * x_out = x_k + (sigmas[step+1] - sigmas[step]) * v with the difference formed
+ * in fp64 on the device ([6B] §1). Invalid pointers or step < 0 return
+ * QI21_ERR_INVALID_ARG before anything is enqueued; the table is not bounds-
+ * checked on the device. */
+qi21_status qi21_modulation_at(const qi21_config *cfg, const qi21_weights *w, const double *sigmas,
+                               int32_t step, double t_per_sigma, float *mod_row, float *scale_final,
+                               void *ws, size_t ws_bytes, void *stream);
+qi21_status qi21_euler_update_at(const float *x_k, const float *v, const double *sigmas, int32_t step,
+                                 float *x_out, int64_t n, void *stream);
+
+/* Whole image ([6B] §4 the 8-step Euler loop; [E2E] §3 extract once, then
+ * cached steps): enqueues, on one stream and with no host synchronisation,
+ *   mod_row_prefix = modulation(t = 0); qi21_prefix_extract;
+ *   for k in [0, n_steps): modulation_at(k) -> mod_row_target, scale_final;
+ *                          qi21_cached_step(x) -> v; x = euler_update_at(k)
+ * so that the whole call can be captured once into a CUDA graph and replayed
+ * per image (make one uncaptured call first: it sets kernel attributes).
+ *   prefix_hidden [B][P][d] f32; cos_sin_prefix [P][Dh/2][2], kv_limit_prefix [P],
+ *   cos_sin_target [N][Dh/2][2]; sigmas [n_steps+1] f64 device;
+ *   x [B][N][C] f32: x_0 in, x_{n_steps} out; v [B][N][C] f32 scratch (last v);
+ *   mod_row_prefix, mod_row_target [chunks*d], scale_final [d] f32 scratch.
+ * All device buffers are the caller's. Stops at the first failing call and
+ * returns its status. */
+qi21_status qi21_denoise_image(const qi21_config *cfg, const qi21_weights *w, qi21_kv_cache *cache,
+                               const float *prefix_hidden, const float *cos_sin_prefix,
+                               const int32_t *kv_limit_prefix, const float *cos_sin_target,
+                               const double *sigmas, int32_t n_steps, double t_per_sigma, float *x,
+                               float *v, float *mod_row_prefix, float *mod_row_target,
+                               float *scale_final, void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronise the stream, then read and clear the device error word of the
  * workspace. Returns QI21_OK, QI21_ERR_DEVICE_TIMEOUT, QI21_ERR_DEVICE_CHECK or
  * QI21_ERR_CUDA. */

@@ -81,6 +81,11 @@ _SIGS = {
     "qi21_full_recompute_step": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), _I32, _I32, _I32,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_size_t, _P]),
     "qi21_euler_update": (_I32, [_P, _P, ct.c_double, ct.c_double, _P, ct.c_int64, _P]),
+    "qi21_modulation_at": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), _P, _I32, ct.c_double, _P,
+                                  _P, _P, ct.c_size_t, _P]),
+    "qi21_euler_update_at": (_I32, [_P, _P, _P, _I32, _P, ct.c_int64, _P]),
+    "qi21_denoise_image": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.POINTER(qi21_kv_cache),
+                                  _P, _P, _P, _P, _P, _I32, ct.c_double, _P, _P, _P, _P, _P, _P, ct.c_size_t, _P]),
     "qi21_check_device_error": (_I32, [_P, ct.c_size_t, _P]),
     "qi21_status_string": (ct.c_char_p, [_I32]),
     "qi21_selftest_wait_timeout": (_I32, [_P, ct.c_size_t, ct.c_int64, _P]),
@@ -223,6 +228,25 @@ def qi21_full_recompute_step(cfg, weights, batch, n_prefix, n_target, prefix_hid
 
 def qi21_euler_update(x_k, v, sigma_k, sigma_k1, x_out, n, stream=0):
     return lib.qi21_euler_update(_addr(x_k), _addr(v), float(sigma_k), float(sigma_k1), _addr(x_out), int(n), stream)
+
+
+def qi21_modulation_at(cfg, weights, sigmas, step, t_per_sigma, mod_row, scale_final, ws, ws_bytes, stream=0):
+    return lib.qi21_modulation_at(ct.byref(cfg), ct.byref(weights), _addr(sigmas), int(step), float(t_per_sigma),
+                                  _addr(mod_row), _addr(scale_final), _addr(ws), ws_bytes, stream)
+
+
+def qi21_euler_update_at(x_k, v, sigmas, step, x_out, n, stream=0):
+    return lib.qi21_euler_update_at(_addr(x_k), _addr(v), _addr(sigmas), int(step), _addr(x_out), int(n), stream)
+
+
+def qi21_denoise_image(cfg, weights, cache, prefix_hidden, cos_sin_prefix, kv_limit_prefix, cos_sin_target,
+                       sigmas, n_steps, t_per_sigma, x, v, mod_row_prefix, mod_row_target, scale_final, ws,
+                       ws_bytes, stream=0):
+    return lib.qi21_denoise_image(ct.byref(cfg), ct.byref(weights), ct.byref(cache), _addr(prefix_hidden),
+                                  _addr(cos_sin_prefix), _addr(kv_limit_prefix), _addr(cos_sin_target),
+                                  _addr(sigmas), int(n_steps), float(t_per_sigma), _addr(x), _addr(v),
+                                  _addr(mod_row_prefix), _addr(mod_row_target), _addr(scale_final), _addr(ws),
+                                  ws_bytes, stream)
 
 
 def qi21_check_device_error(ws, ws_bytes, stream=0):

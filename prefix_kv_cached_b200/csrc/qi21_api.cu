@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <vector>
+#include <type_traits>
 
 #include "qi21.h"
 #include "qi21_internal.h"
@@ -491,53 +492,66 @@ static qi21_status finish(Launcher &L) { return L.status; }
 using namespace qi21;
 
 // ------------------------------------------------------------------ entry points
-extern "C" qi21_status qi21_modulation(const qi21_config *c, const qi21_weights *w, double t, float *mod_row,
-                                       float *scale_final, void *ws, size_t ws_bytes, void *stream) {
+// Modulation rows for the timestep embedding given either on the host
+// (emb != null) or as a device table of sigmas (sigmas[step] * t_per_sigma).
+static qi21_status modulation_impl(const qi21_config *c, const qi21_weights *w, const TembArg *emb,
+                                   const double *sigmas, int step, double t_per_sigma, float *mod_row,
+                                   float *scale_final, void *ws, size_t ws_bytes, void *stream) {
     qi21_status s = check_shapes(c);
     if (s) return s;
     if (!w || !al16(w->w_t1) || !al16(w->w_t2) || !al16(w->w_mod) || !al16(w->w_fin)) return QI21_ERR_INVALID_ARG;
     if (!al16(mod_row) || !al16(scale_final) || !al16(ws)) return QI21_ERR_INVALID_ARG;
-    if (!std::isfinite(t)) return QI21_ERR_INVALID_ARG;
     const WsLayout lay = ws_layout(*c, 1, 0, 1);
     if (ws_bytes < lay.modtmp + align256(sizeof(float) * 2 * c->d_model)) return QI21_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = (cudaStream_t)stream;
     Launcher L(st);
     const int d = c->d_model, K0 = c->time_dim, nch = c->use_shift ? 6 : 4;
-    TembArg emb;
-    qi21_timestep_embedding(t, K0, emb.v);
     float *a1 = (float *)((char *)ws + lay.modtmp), *e = a1 + d;
     const size_t xs = sizeof(float) * d;
-    if (c->dtype == QI21_DTYPE_BF16) {
+    auto run = [&](auto *wt) {
+        using T = std::remove_const_t<std::remove_pointer_t<decltype(wt)>>;
         static bool attr = false;
         if (!attr) {
-            cudaFuncSetAttribute(k_gemv2<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            cudaFuncSetAttribute(k_gemv2<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
             attr = true;
         }
-        L.run("temb_in", [&] { k_temb_in<bf16><<<(d + 7) / 8, 256, 0, st>>>((const bf16 *)w->w_t1, emb, K0, d, a1); });
+        if (emb)
+            L.run("temb_in", [&] { k_temb_in<T><<<(d + 7) / 8, 256, 0, st>>>((const T *)w->w_t1, *emb, K0, d, a1); });
+        else
+            L.run("temb_in", [&] {
+                k_temb_in_sigma<T><<<(d + 7) / 8, 256, 0, st>>>((const T *)w->w_t1, sigmas, step, t_per_sigma, K0, d,
+                                                               a1);
+            });
         L.run("gemv", [&] {
-            k_gemv2<bf16><<<(d + 7) / 8, 256, xs, st>>>((const bf16 *)w->w_t2, d, e, (const bf16 *)w->w_t2, 0, e, a1, d, 0);
+            k_gemv2<T><<<(d + 7) / 8, 256, xs, st>>>((const T *)w->w_t2, d, e, (const T *)w->w_t2, 0, e, a1, d, 0);
         });
         L.run("gemv", [&] {
-            k_gemv2<bf16><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const bf16 *)w->w_mod, nch * d, mod_row,
-                                                                  (const bf16 *)w->w_fin, d, scale_final, e, d, 1);
+            k_gemv2<T><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const T *)w->w_mod, nch * d, mod_row,
+                                                               (const T *)w->w_fin, d, scale_final, e, d, 1);
         });
-    } else {
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(k_gemv2<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-            attr = true;
-        }
-        L.run("temb_in", [&] { k_temb_in<float><<<(d + 7) / 8, 256, 0, st>>>((const float *)w->w_t1, emb, K0, d, a1); });
-        L.run("gemv", [&] {
-            k_gemv2<float><<<(d + 7) / 8, 256, xs, st>>>((const float *)w->w_t2, d, e, (const float *)w->w_t2, 0, e, a1,
-                                                          d, 0);
-        });
-        L.run("gemv", [&] {
-            k_gemv2<float><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const float *)w->w_mod, nch * d, mod_row,
-                                                                   (const float *)w->w_fin, d, scale_final, e, d, 1);
-        });
-    }
+    };
+    if (c->dtype == QI21_DTYPE_BF16)
+        run((const bf16 *)nullptr);
+    else
+        run((const float *)nullptr);
     return finish(L);
+}
+
+extern "C" qi21_status qi21_modulation(const qi21_config *c, const qi21_weights *w, double t, float *mod_row,
+                                       float *scale_final, void *ws, size_t ws_bytes, void *stream) {
+    if (!std::isfinite(t)) return QI21_ERR_INVALID_ARG;
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    TembArg emb;
+    qi21_timestep_embedding(t, c->time_dim, emb.v);
+    return modulation_impl(c, w, &emb, nullptr, 0, 0.0, mod_row, scale_final, ws, ws_bytes, stream);
+}
+
+extern "C" qi21_status qi21_modulation_at(const qi21_config *c, const qi21_weights *w, const double *sigmas,
+                                          int32_t step, double t_per_sigma, float *mod_row, float *scale_final,
+                                          void *ws, size_t ws_bytes, void *stream) {
+    if (!sigmas || ((uintptr_t)sigmas & 7) || step < 0 || !std::isfinite(t_per_sigma)) return QI21_ERR_INVALID_ARG;
+    return modulation_impl(c, w, nullptr, sigmas, step, t_per_sigma, mod_row, scale_final, ws, ws_bytes, stream);
 }
 
 extern "C" qi21_status qi21_prefix_extract(const qi21_config *c, const qi21_weights *w, qi21_kv_cache *cache,
@@ -701,6 +715,44 @@ extern "C" qi21_status qi21_euler_update(const float *x_k, const float *v, doubl
     const float dsig = (float)(sigma_k1 - sigma_k);
     L.run("euler", [&] { k_euler<<<grid_for((n + 3) / 4, 256), 256, 0, st>>>(x_k, v, dsig, x_out, n); });
     return finish(L);
+}
+
+extern "C" qi21_status qi21_euler_update_at(const float *x_k, const float *v, const double *sigmas, int32_t step,
+                                            float *x_out, int64_t n, void *stream) {
+    if (!al16(x_k) || !al16(v) || !al16(x_out) || n < 0) return QI21_ERR_INVALID_ARG;
+    if (!sigmas || ((uintptr_t)sigmas & 7) || step < 0) return QI21_ERR_INVALID_ARG;
+    if (n == 0) return QI21_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    L.run("euler", [&] { k_euler_sigma<<<grid_for((n + 3) / 4, 256), 256, 0, st>>>(x_k, v, sigmas, step, x_out, n); });
+    return finish(L);
+}
+
+extern "C" qi21_status qi21_denoise_image(const qi21_config *c, const qi21_weights *w, qi21_kv_cache *cache,
+                                          const float *prefix_hidden, const float *cos_sin_prefix,
+                                          const int32_t *kv_limit_prefix, const float *cos_sin_target,
+                                          const double *sigmas, int32_t n_steps, double t_per_sigma, float *x,
+                                          float *v, float *mod_row_prefix, float *mod_row_target,
+                                          float *scale_final, void *ws, size_t ws_bytes, void *stream) {
+    if (!cache || n_steps < 1 || !sigmas) return QI21_ERR_INVALID_ARG;
+    int launches = 0;
+    qi21_status s = qi21_modulation(c, w, 0.0, mod_row_prefix, scale_final, ws, ws_bytes, stream);
+    launches += g_last_launches;
+    if (!s) s = qi21_prefix_extract(c, w, cache, prefix_hidden, cos_sin_prefix, kv_limit_prefix, mod_row_prefix, ws,
+                                    ws_bytes, stream);
+    launches += g_last_launches;
+    const int64_t n = (int64_t)cache->batch * cache->n_target * c->latent_ch;
+    for (int k = 0; k < n_steps && !s; ++k) {
+        s = qi21_modulation_at(c, w, sigmas, k, t_per_sigma, mod_row_target, scale_final, ws, ws_bytes, stream);
+        launches += g_last_launches;
+        if (!s) s = qi21_cached_step(c, w, cache, x, cos_sin_target, mod_row_target, scale_final, v, ws, ws_bytes,
+                                     stream);
+        launches += g_last_launches;
+        if (!s) s = qi21_euler_update_at(x, v, sigmas, k, x, n, stream);
+        launches += g_last_launches;
+    }
+    g_last_launches = launches;
+    return s;
 }
 
 extern "C" qi21_status qi21_check_device_error(void *ws, size_t ws_bytes, void *stream) {

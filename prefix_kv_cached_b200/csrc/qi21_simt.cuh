@@ -561,8 +561,8 @@ __global__ void __launch_bounds__(256) k_final64(const float *__restrict__ h, in
 }
 
 // x_out = x + dsig * v  (6B page §1).
-static __global__ void k_euler(const float *__restrict__ x, const float *__restrict__ v, float dsig,
-                        float *__restrict__ xo, int64_t n) {
+__device__ __forceinline__ void euler_body(const float *__restrict__ x, const float *__restrict__ v, float dsig,
+                                           float *__restrict__ xo, int64_t n) {
     const int64_t n4 = n >> 2;
     const float4 *x4 = reinterpret_cast<const float4 *>(x);
     const float4 *v4 = reinterpret_cast<const float4 *>(v);
@@ -574,6 +574,18 @@ static __global__ void k_euler(const float *__restrict__ x, const float *__restr
     for (int64_t i = (n4 << 2) + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x)
         xo[i] = fmaf(dsig, v[i], x[i]);
+}
+
+static __global__ void k_euler(const float *__restrict__ x, const float *__restrict__ v, float dsig,
+                        float *__restrict__ xo, int64_t n) {
+    euler_body(x, v, dsig, xo, n);
+}
+
+// Euler update with the step read from a device table of sigmas; the
+// difference is formed in fp64 and rounded once, as on the host path.
+static __global__ void k_euler_sigma(const float *__restrict__ x, const float *__restrict__ v,
+                                     const double *__restrict__ sigmas, int step, float *__restrict__ xo, int64_t n) {
+    euler_body(x, v, (float)(sigmas[step + 1] - sigmas[step]), xo, n);
 }
 
 // ---------------------------------------------------------------------------
@@ -626,6 +638,31 @@ __global__ void __launch_bounds__(256) k_temb_in(const T *__restrict__ W, TembAr
                                                  float *__restrict__ y) {
     __shared__ float xs[512];
     for (int k = threadIdx.x; k < K; k += blockDim.x) xs[k] = emb.v[k];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (n >= N) return;
+    const float acc = warp_sum(dot_row(W + (size_t)n * K, xs, K, lane));
+    if (lane == 0) y[n] = silu_f(acc);
+}
+
+// As k_temb_in, with the embedding formed on the device from a device table of
+// sigmas (so that a captured sequence of steps reads its sigma at run time):
+// t = t_per_sigma * sigmas[step], emb = [cos(t f_i) | sin(t f_i)],
+// f_i = 10000^(-2i/K), in fp64 rounded once to fp32 (the host helper
+// qi21_timestep_embedding does the same arithmetic).
+template <typename T>
+__global__ void __launch_bounds__(256) k_temb_in_sigma(const T *__restrict__ W, const double *__restrict__ sigmas,
+                                                       int step, double t_per_sigma, int K, int N,
+                                                       float *__restrict__ y) {
+    __shared__ float xs[512];
+    const int half = K / 2;
+    const double t = t_per_sigma * sigmas[step];
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+        const double f = pow(10000.0, -2.0 * i / K);
+        xs[i] = (float)cos(t * f);
+        xs[half + i] = (float)sin(t * f);
+    }
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int n = blockIdx.x * 8 + (threadIdx.x >> 5);

@@ -122,6 +122,40 @@ class Qi21Runner:
     def euler(self, x: torch.Tensor, v: torch.Tensor, s0: float, s1: float, x_out: torch.Tensor):
         B.check("qi21_euler_update", B.qi21_euler_update(x, v, s0, s1, x_out, x.numel(), self.stream))
 
+    # ------------------------------------------------------------------ whole image
+    # t = 1000 * sigma (3B page §1; 6B page §3)
+    T_PER_SIGMA = 1000.0
+
+    def denoise_image(self, prefix_hidden: torch.Tensor, x: torch.Tensor, sigmas_dev: torch.Tensor,
+                      v: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """One call of qi21_denoise_image: extract, then len(sigmas_dev) - 1 cached
+        steps with Euler, all enqueued on the current stream; x is updated in
+        place (x_0 in, final latent out). sigmas_dev: float64 device tensor."""
+        assert sigmas_dev.dtype == torch.float64 and sigmas_dev.is_cuda and sigmas_dev.numel() >= 2
+        v = torch.empty_like(x) if v is None else v
+        B.check("qi21_denoise_image", B.qi21_denoise_image(
+            self.cfg, self.wstruct, self.cache, prefix_hidden, self.cos_sin_prefix, self.kv_limit_prefix,
+            self.cos_sin_target, sigmas_dev, sigmas_dev.numel() - 1, self.T_PER_SIGMA, x, v, self.mod_prefix,
+            self.mod_target, self.scale_final, self.ws, self.ws_bytes, self.stream))
+        return x
+
+    def capture_image(self, prefix_hidden: torch.Tensor, x: torch.Tensor, sigmas_dev: torch.Tensor):
+        """Capture the whole-image call into a CUDA graph (after one eager call
+        that sets kernel attributes). Replaying the returned graph re-runs the
+        image on the current contents of prefix_hidden, x and sigmas_dev."""
+        v = torch.empty_like(x)
+        x_warm = x.clone()
+        self.denoise_image(prefix_hidden, x_warm, sigmas_dev, v)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+                self.denoise_image(prefix_hidden, x, sigmas_dev, v)
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        return g
+
     def check_device(self):
         B.check("qi21_check_device_error", B.qi21_check_device_error(self.ws, self.ws_bytes, self.stream))
 

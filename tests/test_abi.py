@@ -128,6 +128,22 @@ def test_host_validation_returns_before_launch(B):
     assert B.qi21_full_recompute_step(cfg, w, 0, 8, 4, fake, fake, fake, fake, fake, fake, fake, fake, fake,
                                       ws_bytes, 0) == B.QI21_ERR_SHAPE
     assert B.qi21_euler_update(fake, fake, 1.0, float("nan"), fake, 4, 0) == B.QI21_ERR_INVALID_ARG
+    # device-indexed forms and the whole-image call: bad sigma tables, steps and configs
+    mod = fake
+    assert B.qi21_modulation_at(cfg, w, 0, 0, 1000.0, mod, mod, fake, ws_bytes, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_modulation_at(cfg, w, fake + 4, 0, 1000.0, mod, mod, fake, ws_bytes, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_modulation_at(cfg, w, fake, -1, 1000.0, mod, mod, fake, ws_bytes, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_modulation_at(bad, w, fake, 0, 1000.0, mod, mod, fake, ws_bytes, 0) == B.QI21_ERR_SHAPE
+    assert B.qi21_euler_update_at(fake, fake, fake, -1, fake, 4, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_euler_update_at(fake + 4, fake, fake, 0, fake, 4, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_euler_update_at(fake, fake, 0, 0, fake, 4, 0) == B.QI21_ERR_INVALID_ARG
+    args = (fake, fake, fake, fake)
+    assert B.qi21_denoise_image(cfg, w, cache, *args, fake, 0, 1000.0, fake, fake, mod, mod, mod, fake, ws_bytes,
+                                0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_denoise_image(cfg, w, cache, *args, 0, 8, 1000.0, fake, fake, mod, mod, mod, fake, ws_bytes,
+                                0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_denoise_image(bad, w, cache, *args, fake, 8, 1000.0, fake, fake, mod, mod, mod, fake, ws_bytes,
+                                0) == B.QI21_ERR_SHAPE
     assert B.qi21_status_string(B.QI21_ERR_DEVICE_TIMEOUT).startswith("device wait")
 
 
