@@ -99,10 +99,25 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
 
 
-def kernel_source_hash():
+# The files a kernel's code and launch configuration come from: a stored ncu
+# figure stays valid while these are unchanged.
+_COMMON_SOURCES = ("qi21_common.cuh", "qi21_sm100.cuh", "qi21_internal.h", "qi21_api.cu")
+KERNEL_SOURCES = {
+    "attn": ("qi21_attn_tc.cuh",) + _COMMON_SOURCES,
+    "gemm_qkv": ("qi21_gemm_tc.cuh",) + _COMMON_SOURCES,
+    "gemm_o": ("qi21_gemm_tc.cuh",) + _COMMON_SOURCES,
+    "gemm_gateup": ("qi21_gemm_tc.cuh",) + _COMMON_SOURCES,
+    "gemm_down": ("qi21_gemm_tc.cuh",) + _COMMON_SOURCES,
+}
+
+
+def kernel_source_hash(kernel=None):
+    """sha256 (16 hex digits) of the kernel's source files (all of csrc/ when
+    kernel is None or unknown)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "prefix_kv_cached_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc))
+    for f in names:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -110,14 +125,14 @@ def kernel_source_hash():
 
 def load_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the kernel's current sources (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
     e = j.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
