@@ -78,18 +78,31 @@ def _gelu_tanh(x):
     return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
 
 
-def prefix_tokens(w, demo_rgba: np.ndarray) -> np.ndarray:
-    """The lab's 7 prefix rows: txt_in(text slots) and img_in(cond latent) + slot vector.
+def text_slot_tokens(w) -> np.ndarray:
+    """Lab [1B]: the text slots 0, 1, 3 of the VLM context -> zero-centred RMSNorm -> GELU MLP."""
+    return np.stack([_gelu_tanh(O.rmsnorm_zero_centre(w["context"][i], w["rms_ctx"], EPS) @ w["w_txt1"])
+                     @ w["w_txt2"] for i in (0, 1, 3)])
 
-    Lab [1A]: cond latent = standardise(rgba W_enc + b_enc); lab [1B]: text slot
-    -> zero-centred RMSNorm -> GELU MLP; lab [2A]: the image slot vector is
-    added to each of its 4 img_in tokens.
-    """
+
+def cond_image_tokens(w, demo_rgba: np.ndarray) -> np.ndarray:
+    """Lab [1A]: cond latent = standardise(rgba W_enc + b_enc), then img_in (4 tokens)."""
     z = np.asarray(demo_rgba, dtype=np.float64).reshape(-1, RGBA) @ w["w_enc"] + w["b_enc"]
     z_std = (z - w["latent_mean"]) / w["latent_std"]
-    cond = z_std @ w["w_img_in"] + w["context"][2]
-    txt = np.stack([_gelu_tanh(O.rmsnorm_zero_centre(w["context"][i], w["rms_ctx"], EPS)
-                               @ w["w_txt1"]) @ w["w_txt2"] for i in (0, 1, 3)])
+    return z_std @ w["w_img_in"]
+
+
+def slot_vectors(w) -> np.ndarray:
+    """The 4 VLM slots as the packing reads them: txt_in of the text slots, the
+    image slot (index 2) as the VLM left it (lab [1B], [2A])."""
+    txt = text_slot_tokens(w)
+    return np.stack([txt[0], txt[1], w["context"][2], txt[2]])
+
+
+def prefix_tokens(w, demo_rgba: np.ndarray) -> np.ndarray:
+    """The lab's 7 prefix rows, laid out as the lab does it: two text rows, the
+    image slot vector added to each of the 4 img_in tokens, the last text row."""
+    txt = text_slot_tokens(w)
+    cond = cond_image_tokens(w, demo_rgba) + w["context"][2]
     return np.concatenate([txt[:2], cond, txt[2:]], axis=0)
 
 

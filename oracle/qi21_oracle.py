@@ -37,7 +37,14 @@ reason in the design notes of the repository):
   (lab [3B]);
 * RoPE pairs are adjacent dims (2j, 2j+1), angle = sum over axes of coord * omega
   (lab [3A]); image grids are centred with integer n//2 (lab [3A], End-to-end
-  lab §3); text tokens take (i, i, i) counting text tokens only.
+  lab §3); text tokens take (i, i, i) counting text tokens only;
+* joint packing of the prefix values: every VLM image slot stands for
+  IMG_TOKENS_PER_SLOT = 4 latent cells (2A page), so an image of h*w cells
+  (h*w divisible by 4) has h*w/4 slots; repeat_interleave writes each slot's
+  vector at 4 consecutive positions of the image's token run (raster order).
+  At image positions the 2A page replaces the slot value by the img_in token
+  (the default, PACK_SUBSTITUTE); the lab adds the two (its COND_TOKENS,
+  PACK_ADD).
 
 Parity unpinned: nothing. Each function has a pin in ``tests/test_oracle_pins.py``
 (page-printed values, closed forms, library routines or brute force).
@@ -110,6 +117,57 @@ def rope_coords(segments, frame_mode: int = 0) -> np.ndarray:
                     coords.append((f, r - a // 2, c - b // 2))
             img += 1
     return np.array(coords, dtype=np.int64)
+
+
+# Joint packing of the prefix values (2A page; lab [2A])
+IMG_TOKENS_PER_SLOT = 4        # 2A page: one VLM image slot <-> a 2x2 block of latent cells
+PACK_SUBSTITUTE = 0            # 2A page, mechanism (2): img_in replaces the slot value
+PACK_ADD = 1                   # lab [2A]: COND_TOKENS = img_in(latent) + image slot vector
+
+
+def slot_expansion(segments):
+    """Index tables of the 4x slot expansion over the prefix (every segment but
+    the last, which is the target).
+
+    2A page, mechanism (1): repeat_interleave repeats each VLM slot vector
+    consecutively, once for a text slot and IMG_TOKENS_PER_SLOT times for an
+    image slot (repeats = where(img_mask, 4, 1)); (2): image positions take the
+    img_in token of their latent cell. Returns slot_of int64[P] (the slot each
+    prefix token expands), img_row int64[P] (row of the table of image tokens,
+    reference images concatenated in order, raster order inside an image; -1 at
+    text positions), n_slots and n_img.
+    """
+    repeats: List[int] = []
+    img_row: List[int] = []
+    n_img = 0
+    for kind, a, b in segments[:-1]:
+        if kind == SEG_TEXT:
+            repeats += [1] * a
+            img_row += [-1] * a
+        else:
+            cells = a * b
+            if cells % IMG_TOKENS_PER_SLOT:
+                raise ValueError("an image slot covers 4 latent cells: h*w must be divisible by 4")
+            repeats += [IMG_TOKENS_PER_SLOT] * (cells // IMG_TOKENS_PER_SLOT)
+            img_row += list(range(n_img, n_img + cells))
+            n_img += cells
+    slot_of = np.repeat(np.arange(len(repeats), dtype=np.int64), repeats)
+    return slot_of, np.array(img_row, dtype=np.int64), len(repeats), n_img
+
+
+def pack_prefix(ctx: np.ndarray, img_tokens: np.ndarray, segments, mode: int = PACK_SUBSTITUTE) -> np.ndarray:
+    """Prefix hidden states [P, d] from the VLM slot vectors ctx [n_slots, d]
+    (text slots after txt_in, image slots as the VLM left them) and the img_in
+    tokens of the reference images img_tokens [n_img, d] (2A page, mechanism
+    (1)-(2); lab [2A])."""
+    slot_of, img_row, _, _ = slot_expansion(segments)
+    out = ctx[slot_of].copy()
+    m = img_row >= 0
+    if mode == PACK_SUBSTITUTE:
+        out[m] = img_tokens[img_row[m]]
+    else:
+        out[m] = out[m] + img_tokens[img_row[m]]
+    return out
 
 
 def block_causal_allowed(image_ids: np.ndarray) -> np.ndarray:

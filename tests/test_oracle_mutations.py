@@ -85,3 +85,30 @@ def test_euler_sign_mutation_caught(monkeypatch):
     for k in range(8):
         x = O.euler_step(x, v, sig[k], sig[k + 1])
     assert not np.allclose(x, x0 - v)
+
+
+PACK_MUTATIONS = [
+    ("slot_expansion", "repeats += [IMG_TOKENS_PER_SLOT] * (cells // IMG_TOKENS_PER_SLOT)",
+     "repeats += [1] * (cells // IMG_TOKENS_PER_SLOT)"),                                  # no 4x expansion
+    ("slot_expansion", "img_row += list(range(n_img, n_img + cells))",
+     "img_row += list(range(n_img + cells - 1, n_img - 1, -1))"),                         # cells reversed
+    ("pack_prefix", "out[m] = img_tokens[img_row[m]]", "out[m] = out[m] + img_tokens[img_row[m]]"),  # add
+    ("pack_prefix", "out[m] = out[m] + img_tokens[img_row[m]]", "out[m] = img_tokens[img_row[m]]"),  # replace
+]
+
+
+@pytest.mark.parametrize("fname,old,new", PACK_MUTATIONS, ids=[f"{m[0]}:{i}" for i, m in enumerate(PACK_MUTATIONS)])
+def test_packing_pins_catch_mutation(monkeypatch, fname, old, new):
+    from tests import test_oracle_pins as P
+    from tests.conftest import load_golden as lg
+    monkeypatch.setattr(O, fname, _mutant(getattr(O, fname), old, new))
+    pins = [lambda: P.test_slot_expansion_matches_page_repeats(lg), P.test_packed_length_formula,
+            P.test_slot_expansion_brute_force, lambda: P.test_pack_add_reproduces_the_lab_prefix_rows(lg),
+            P.test_pack_substitute_takes_img_in_at_image_positions]
+    failed = 0
+    for pin in pins:
+        try:
+            pin()
+        except (AssertionError, IndexError, ValueError):   # a pin that fails or breaks catches it
+            failed += 1
+    assert failed > 0, f"mutation in {fname} not caught by any packing pin"

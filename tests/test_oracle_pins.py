@@ -370,3 +370,92 @@ def test_velocity_depends_on_sigma():
         vs.append(O.cached_step(model, seq, ck, cv, x0[0], mt, sf)[0])
     for a, b in itertools.combinations(vs, 2):
         assert np.max(np.abs(a - b)) > 1e-8
+
+
+# ---------------------------------------------------------------------------- joint packing (2A page)
+def _random_layouts(n=20, seed=5):
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        segs = []
+        for _ in range(rng.integers(1, 5)):
+            if rng.random() < 0.5:
+                segs.append((O.SEG_TEXT, int(rng.integers(1, 6)), 0))
+            else:
+                segs.append((O.SEG_IMAGE, 2 * int(rng.integers(1, 4)), 2 * int(rng.integers(1, 4))))
+        segs.append((O.SEG_IMAGE, 2, 2))                        # target last
+        out.append(segs)
+    return out
+
+
+def test_slot_expansion_matches_page_repeats(golden):
+    """Lab page 1:1 table, row 2A: repeats = [1, 1, 4, 1] over the slots [text, text, image, text]."""
+    g = golden("toy_sequence.json")
+    slot_of, img_row, n_slots, n_img = O.slot_expansion([tuple(s) for s in g["segments"]])
+    assert slot_of.tolist() == np.repeat(np.arange(4), g["repeats"]).tolist()
+    assert img_row.tolist() == [-1, -1, 0, 1, 2, 3, -1]
+    assert (n_slots, n_img, len(slot_of)) == (4, 4, g["P"])
+
+
+def test_packed_length_formula():
+    """2A page: length = text tokens + 4 x (image slots), and the packing covers exactly the prefix."""
+    for segs in _random_layouts():
+        slot_of, img_row, n_slots, n_img = O.slot_expansion(segs)
+        n_text = sum(a for k, a, _ in segs[:-1] if k == O.SEG_TEXT)
+        image_slots = sum(a * b // 4 for k, a, b in segs[:-1] if k == O.SEG_IMAGE)
+        assert len(slot_of) == n_text + 4 * image_slots == O.token_metadata(segs)[3]
+        assert n_slots == n_text + image_slots and n_img == 4 * image_slots
+
+
+def test_slot_expansion_brute_force():
+    """Walk the prefix position by position: a text token takes the next slot; an
+    image takes the next slot every 4 cells and the next image-token row every cell."""
+    for segs in _random_layouts():
+        want_slot, want_row = [], []
+        slot = row = 0
+        for kind, a, b in segs[:-1]:
+            if kind == O.SEG_TEXT:
+                for _ in range(a):
+                    want_slot.append(slot)
+                    want_row.append(-1)
+                    slot += 1
+            else:
+                for cell in range(a * b):
+                    want_slot.append(slot + cell // 4)
+                    want_row.append(row)
+                    row += 1
+                slot += a * b // 4
+        slot_of, img_row, _, _ = O.slot_expansion(segs)
+        assert slot_of.tolist() == want_slot and img_row.tolist() == want_row
+
+
+def test_pack_add_reproduces_the_lab_prefix_rows(golden):
+    """Lab [2A]: PREFIX_TOKENS = [txt0, txt1, img_in(cond) + slot2, txt3] — built there by concatenation."""
+    g = golden("lab_checks.json")
+    w = LR.draw_lab_weights()
+    demo = np.array(g["demo_rgba"])
+    segs = [tuple(s) for s in golden("toy_sequence.json")["segments"]]
+    got = O.pack_prefix(LR.slot_vectors(w), LR.cond_image_tokens(w, demo), segs, O.PACK_ADD)
+    assert np.array_equal(got, LR.prefix_tokens(w, demo))
+
+
+def test_pack_substitute_takes_img_in_at_image_positions():
+    """2A page, mechanism (2): image positions hold the img_in token of their cell, text positions their slot."""
+    rng = np.random.default_rng(8)
+    for segs in _random_layouts(8):
+        slot_of, img_row, n_slots, n_img = O.slot_expansion(segs)
+        ctx = rng.standard_normal((n_slots, 6))
+        img = rng.standard_normal((n_img, 6))
+        out = O.pack_prefix(ctx, img, segs, O.PACK_SUBSTITUTE)
+        pos = 0
+        for kind, a, b in segs[:-1]:
+            n = a if kind == O.SEG_TEXT else a * b
+            for t in range(n):
+                if kind == O.SEG_TEXT:
+                    assert np.array_equal(out[pos], ctx[slot_of[pos]])
+                else:
+                    assert np.array_equal(out[pos], img[img_row[pos]])
+                pos += 1
+        image_slots = set(slot_of[img_row >= 0].tolist())
+        for s_ in image_slots:                       # an image slot's own vector never survives
+            assert not any(np.array_equal(r, ctx[s_]) for r in out)
