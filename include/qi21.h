@@ -148,7 +148,26 @@ qi21_status qi21_rope_omega_axial(int32_t head_dim, double base, double *omega);
 qi21_status qi21_rope_table(int32_t head_dim, const int32_t *coords, int32_t S,
                             const double *omega, float *cos_sin);
 
-/* Sin-cos timestep embedding [time_dim] (host, fp64 math, float result):
+/* Latent cells per VLM image slot: one slot stands for a 2x2 block ([2A]). */
+#define QI21_IMG_TOKENS_PER_SLOT 4
+
+/* Index tables of the joint packing of the prefix values ([2A] mechanisms (1)
+ * and (2); [LAB] 2A repeats = where(img_mask, 4, 1)). Host-only and pure.
+ * Over the prefix (every segment but the last, the target): a text token is
+ * one VLM slot; an image of h*w latent cells (h*w divisible by 4) has h*w/4
+ * slots, each written at 4 consecutive positions of the image's run.
+ *   slot_of [P]: the slot each prefix token expands (index into ctx rows)
+ *   img_row [P]: row of the img_in token table at image positions (reference
+ *                images in order, raster order inside each), -1 at text positions
+ * Host arrays of capacity entries, either may be NULL; pass both NULL to query
+ * P, n_slots (rows of ctx) and n_img (rows of the img_in token table).
+ * Returns QI21_ERR_METADATA for an empty segment, an image whose cell count is
+ * not a multiple of 4, a last segment that is not an image, or capacity < P. */
+qi21_status qi21_build_packing(const qi21_segment *segments, int32_t n_segments, int32_t capacity,
+                               int32_t *slot_of, int32_t *img_row, int32_t *P,
+                               int32_t *n_slots, int32_t *n_img);
+
+/* Sin-cos timestep embedding [time_dim]/* Sin-cos timestep embedding [time_dim] (host, fp64 math, float result):
  * [cos(t f_i) ..., sin(t f_i) ...], f_i = 10000^(-2i/time_dim), t = 1000*sigma
  * ([LAB] 3B, [3B] §1). */
 qi21_status qi21_timestep_embedding(double t, int32_t time_dim, float *emb);
@@ -249,7 +268,32 @@ qi21_status qi21_full_recompute_step(const qi21_config *cfg, const qi21_weights 
 qi21_status qi21_euler_update(const float *x_k, const float *v, double sigma_k, double sigma_k1,
                               float *x_out, int64_t n, void *stream);
 
-/* Device-indexed forms for captured sequences (CUDA graphs): the sigma of a
+/* Joint packing of the prefix values on the device ([2A] mechanisms (1)-(2);
+ * [LAB] 2A). For item b and prefix token s:
+ *   mode QI21_PACK_SUBSTITUTE (the 2A page): out = img_row[s] >= 0 ?
+ *       img_tokens[b][img_row[s]] : ctx[b][slot_of[s]]
+ *   mode QI21_PACK_ADD (the lab's COND_TOKENS): out = ctx[b][slot_of[s]]
+ *       (+ img_tokens[b][img_row[s]] at image positions, one float32 add)
+ *   ctx [B][n_slots][d] f32 device: VLM slot vectors (text slots after txt_in)
+ *   img_tokens [B][n_img][d] f32 device: img_in tokens of the reference images
+ *   slot_of, img_row [P] int32 device (from qi21_build_packing; the indices
+ *       are trusted: they must lie in [0, n_slots) and [-1, n_img))
+ *   out [B][P][d] f32 device: prefix_hidden for qi21_prefix_extract.
+ * Pure data movement (plus the add): bit-exact. Returns QI21_ERR_INVALID_ARG
+ * for null or misaligned pointers, d % 4 != 0 or a bad mode. */
+#define QI21_PACK_SUBSTITUTE 0
+#define QI21_PACK_ADD 1
+qi21_status qi21_pack_prefix(int32_t batch, int32_t P, int32_t d, int32_t n_slots, int32_t n_img,
+                             const float *ctx, const float *img_tokens, const int32_t *slot_of,
+                             const int32_t *img_row, int32_t mode, float *out, void *stream);
+
+/* img_in of latents on the device ([LAB] 1A, patch size 1): out [rows][d] f32 =
+ * latents [rows][C] f32 x w_img_in^T, the projection the cached step applies to
+ * the target latent; here for the reference images' latents before packing. */
+qi21_status qi21_img_in_tokens(const qi21_config *cfg, const qi21_weights *w, const float *latents,
+                               int32_t rows, float *out, void *stream);
+
+/* Device-indexed forms for captured sequences (CUDA graphs)/* Device-indexed forms for captured sequences (CUDA graphs): the sigma of a
  * step is read on the device from sigmas, a table of float64 values in device
  * memory (8-byte aligned, caller-owned, at least step + 2 entries), so one
  * captured sequence serves any sigma schedule written into the table before a

@@ -81,6 +81,10 @@ _SIGS = {
     "qi21_full_recompute_step": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), _I32, _I32, _I32,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _P, ct.c_size_t, _P]),
     "qi21_euler_update": (_I32, [_P, _P, ct.c_double, ct.c_double, _P, ct.c_int64, _P]),
+    "qi21_build_packing": (_I32, [ct.POINTER(qi21_segment), _I32, _I32, _P, _P, ct.POINTER(_I32),
+                                  ct.POINTER(_I32), ct.POINTER(_I32)]),
+    "qi21_pack_prefix": (_I32, [_I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _I32, _P, _P]),
+    "qi21_img_in_tokens": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), _P, _I32, _P, _P]),
     "qi21_modulation_at": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), _P, _I32, ct.c_double, _P,
                                   _P, _P, ct.c_size_t, _P]),
     "qi21_euler_update_at": (_I32, [_P, _P, _P, _I32, _P, ct.c_int64, _P]),
@@ -228,6 +232,37 @@ def qi21_full_recompute_step(cfg, weights, batch, n_prefix, n_target, prefix_hid
 
 def qi21_euler_update(x_k, v, sigma_k, sigma_k1, x_out, n, stream=0):
     return lib.qi21_euler_update(_addr(x_k), _addr(v), float(sigma_k), float(sigma_k1), _addr(x_out), int(n), stream)
+
+
+QI21_PACK_SUBSTITUTE = 0
+QI21_PACK_ADD = 1
+
+
+def qi21_build_packing(segments):
+    """Host index tables of the 4x slot expansion: dict(slot_of, img_row int32[P], P, n_slots, n_img)."""
+    import numpy as np
+    arr = (qi21_segment * len(segments))(*[qi21_segment(int(k), int(a) if k == QI21_SEG_TEXT else 0,
+                                                       int(a) if k == QI21_SEG_IMAGE else 0,
+                                                       int(b) if k == QI21_SEG_IMAGE else 0)
+                                           for (k, a, b) in segments])
+    P, ns, ni = _I32(), _I32(), _I32()
+    check("qi21_build_packing", lib.qi21_build_packing(arr, len(segments), 0, None, None, ct.byref(P),
+                                                       ct.byref(ns), ct.byref(ni)))
+    slot_of = np.zeros(P.value, dtype=np.int32)
+    img_row = np.zeros(P.value, dtype=np.int32)
+    check("qi21_build_packing", lib.qi21_build_packing(arr, len(segments), P.value, slot_of.ctypes.data,
+                                                       img_row.ctypes.data, ct.byref(P), ct.byref(ns),
+                                                       ct.byref(ni)))
+    return {"slot_of": slot_of, "img_row": img_row, "P": P.value, "n_slots": ns.value, "n_img": ni.value}
+
+
+def qi21_pack_prefix(batch, P, d, n_slots, n_img, ctx, img_tokens, slot_of, img_row, mode, out, stream=0):
+    return lib.qi21_pack_prefix(int(batch), int(P), int(d), int(n_slots), int(n_img), _addr(ctx),
+                                _addr(img_tokens), _addr(slot_of), _addr(img_row), int(mode), _addr(out), stream)
+
+
+def qi21_img_in_tokens(cfg, weights, latents, rows, out, stream=0):
+    return lib.qi21_img_in_tokens(ct.byref(cfg), ct.byref(weights), _addr(latents), int(rows), _addr(out), stream)
 
 
 def qi21_modulation_at(cfg, weights, sigmas, step, t_per_sigma, mod_row, scale_final, ws, ws_bytes, stream=0):

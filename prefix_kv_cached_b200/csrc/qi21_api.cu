@@ -717,6 +717,36 @@ extern "C" qi21_status qi21_euler_update(const float *x_k, const float *v, doubl
     return finish(L);
 }
 
+extern "C" qi21_status qi21_pack_prefix(int32_t B, int32_t P, int32_t d, int32_t n_slots, int32_t n_img,
+                                        const float *ctx, const float *img_tokens, const int32_t *slot_of,
+                                        const int32_t *img_row, int32_t mode, float *out, void *stream) {
+    if (B <= 0 || P <= 0 || d <= 0 || d % 4 || n_slots <= 0 || n_img < 0) return QI21_ERR_INVALID_ARG;
+    if (mode != QI21_PACK_SUBSTITUTE && mode != QI21_PACK_ADD) return QI21_ERR_INVALID_ARG;
+    if (!al16(ctx) || !al16(out) || !slot_of || !img_row || (n_img > 0 && !al16(img_tokens)))
+        return QI21_ERR_INVALID_ARG;
+    if ((int64_t)B > 65535) return QI21_ERR_SHAPE;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    L.run("pack", [&] {
+        k_pack_prefix<<<dim3(P, B), 256, 0, st>>>(ctx, img_tokens, slot_of, img_row, P, d, n_slots, n_img, mode, out);
+    });
+    return finish(L);
+}
+
+extern "C" qi21_status qi21_img_in_tokens(const qi21_config *c, const qi21_weights *w, const float *latents,
+                                          int32_t rows, float *out, void *stream) {
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    if (!w || !al16(w->w_img_in) || !al16(latents) || !al16(out) || rows <= 0) return QI21_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L(st);
+    if (c->dtype == QI21_DTYPE_BF16)
+        launch_img_in<bf16>(L, *c, latents, w->w_img_in, out, 1, rows, rows, 0);
+    else
+        launch_img_in<float>(L, *c, latents, w->w_img_in, out, 1, rows, rows, 0);
+    return finish(L);
+}
+
 extern "C" qi21_status qi21_euler_update_at(const float *x_k, const float *v, const double *sigmas, int32_t step,
                                             float *x_out, int64_t n, void *stream) {
     if (!al16(x_k) || !al16(v) || !al16(x_out) || n < 0) return QI21_ERR_INVALID_ARG;

@@ -106,6 +106,57 @@ extern "C" qi21_status qi21_timestep_embedding(double t, int32_t time_dim, float
     return QI21_OK;
 }
 
+extern "C" qi21_status qi21_build_packing(const qi21_segment *seg, int32_t n_seg, int32_t capacity,
+                                          int32_t *slot_of, int32_t *img_row, int32_t *P_out,
+                                          int32_t *n_slots_out, int32_t *n_img_out) {
+    // 2A page, mechanisms (1) and (2): each text token is one VLM slot; an image of
+    // h*w latent cells has h*w/4 slots, each repeated at 4 consecutive positions
+    // (repeat_interleave); image positions also index the table of img_in tokens
+    // (reference images in order, raster order inside an image).
+    if (!seg || n_seg <= 0) return QI21_ERR_INVALID_ARG;
+    if (seg[n_seg - 1].kind != QI21_SEG_IMAGE) return QI21_ERR_METADATA;
+    int64_t P = 0, slots = 0, cells_total = 0;
+    for (int i = 0; i < n_seg - 1; ++i) {
+        if (seg[i].kind == QI21_SEG_TEXT) {
+            if (seg[i].n_text <= 0) return QI21_ERR_METADATA;
+            P += seg[i].n_text;
+            slots += seg[i].n_text;
+        } else if (seg[i].kind == QI21_SEG_IMAGE) {
+            if (seg[i].h <= 0 || seg[i].w <= 0) return QI21_ERR_METADATA;
+            const int64_t cells = (int64_t)seg[i].h * seg[i].w;
+            if (cells % QI21_IMG_TOKENS_PER_SLOT) return QI21_ERR_METADATA;
+            P += cells;
+            slots += cells / QI21_IMG_TOKENS_PER_SLOT;
+            cells_total += cells;
+        } else {
+            return QI21_ERR_INVALID_ARG;
+        }
+    }
+    if (P > INT32_MAX / 4) return QI21_ERR_SHAPE;
+    if (P_out) *P_out = (int32_t)P;
+    if (n_slots_out) *n_slots_out = (int32_t)slots;
+    if (n_img_out) *n_img_out = (int32_t)cells_total;
+    if (!slot_of && !img_row) return QI21_OK;
+    if (capacity < P) return QI21_ERR_METADATA;
+    int64_t pos = 0, slot = 0, row = 0;
+    for (int i = 0; i < n_seg - 1; ++i) {
+        if (seg[i].kind == QI21_SEG_TEXT) {
+            for (int t = 0; t < seg[i].n_text; ++t, ++pos, ++slot) {
+                if (slot_of) slot_of[pos] = (int32_t)slot;
+                if (img_row) img_row[pos] = -1;
+            }
+        } else {
+            const int64_t cells = (int64_t)seg[i].h * seg[i].w;
+            for (int64_t c = 0; c < cells; ++c, ++pos, ++row) {
+                if (slot_of) slot_of[pos] = (int32_t)(slot + c / QI21_IMG_TOKENS_PER_SLOT);
+                if (img_row) img_row[pos] = (int32_t)row;
+            }
+            slot += cells / QI21_IMG_TOKENS_PER_SLOT;
+        }
+    }
+    return QI21_OK;
+}
+
 extern "C" const char *qi21_status_string(qi21_status s) {
     switch (s) {
         case QI21_OK: return "ok";

@@ -561,6 +561,37 @@ __global__ void __launch_bounds__(256) k_final64(const float *__restrict__ h, in
 }
 
 // x_out = x + dsig * v  (6B page §1).
+// Joint packing of the prefix values (2A page, mechanisms (1)-(2)): one block
+// per (prefix token, item) copies its slot vector (text) or its img_in token
+// (image, mode 0) — or adds the two (mode 1, the lab's COND_TOKENS) — with
+// 16-byte loads. Rows whose index tables point outside ctx / img are skipped.
+static __global__ void k_pack_prefix(const float *__restrict__ ctx, const float *__restrict__ img,
+                                     const int32_t *__restrict__ slot_of, const int32_t *__restrict__ img_row,
+                                     int P, int d, int n_slots, int n_img, int mode, float *__restrict__ out) {
+    const int s = blockIdx.x, b = blockIdx.y;
+    const int slot = slot_of[s], ir = img_row[s];
+    if (slot < 0 || slot >= n_slots || ir < -1 || ir >= n_img) return;
+    const float4 *c4 = reinterpret_cast<const float4 *>(ctx + ((size_t)b * n_slots + slot) * d);
+    const float4 *i4 = ir >= 0 ? reinterpret_cast<const float4 *>(img + ((size_t)b * n_img + ir) * d) : nullptr;
+    float4 *o4 = reinterpret_cast<float4 *>(out + ((size_t)b * P + s) * d);
+    for (int i = threadIdx.x; i < d / 4; i += blockDim.x) {
+        float4 v;
+        if (mode == 0) {
+            v = i4 ? i4[i] : c4[i];
+        } else {
+            v = c4[i];
+            if (i4) {
+                const float4 t = i4[i];
+                v.x += t.x;
+                v.y += t.y;
+                v.z += t.z;
+                v.w += t.w;
+            }
+        }
+        o4[i] = v;
+    }
+}
+
 __device__ __forceinline__ void euler_body(const float *__restrict__ x, const float *__restrict__ v, float dsig,
                                            float *__restrict__ xo, int64_t n) {
     const int64_t n4 = n >> 2;

@@ -167,3 +167,31 @@ def test_workspace_covers_the_selected_kernel_family(B):
     finally:
         B.qi21_set_tensor_cores(1)
     assert B.qi21_workspace_bytes(cfg, 2, 198, 300) == tc_bytes
+
+
+def test_packing_tables_bit_exact_vs_oracle(B):
+    from tests.test_oracle_pins import _random_layouts
+    layouts = _random_layouts(30, seed=11) + [[(0, 2, 0), (1, 2, 2), (0, 1, 0), (1, 2, 2)]]
+    for segs in layouts:
+        got = B.qi21_build_packing(segs)
+        slot_of, img_row, n_slots, n_img = O.slot_expansion(segs)
+        assert got["slot_of"].tolist() == slot_of.tolist()
+        assert got["img_row"].tolist() == img_row.tolist()
+        assert (got["P"], got["n_slots"], got["n_img"]) == (len(slot_of), n_slots, n_img)
+
+
+def test_packing_errors_and_validation(B):
+    for segs in ([(0, 3, 0), (1, 3, 3), (1, 2, 2)],      # 9 cells: not whole slots
+                 [(1, 2, 2), (0, 3, 0)]):                 # target is not an image
+        with pytest.raises(B.Qi21Error) as e:
+            B.qi21_build_packing(segs)
+        assert e.value.status == B.QI21_ERR_METADATA
+    fake = 0x10000
+    assert B.qi21_pack_prefix(1, 7, 6, 4, 4, fake, fake, fake, fake, 0, fake, 0) == B.QI21_ERR_INVALID_ARG  # d % 4
+    assert B.qi21_pack_prefix(1, 7, 8, 4, 4, fake, fake, fake, fake, 2, fake, 0) == B.QI21_ERR_INVALID_ARG  # mode
+    assert B.qi21_pack_prefix(1, 7, 8, 4, 4, fake + 4, fake, fake, fake, 0, fake, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_pack_prefix(1, 7, 8, 4, 4, fake, fake, 0, fake, 0, fake, 0) == B.QI21_ERR_INVALID_ARG
+    cfg = _cfg(B)
+    w = B.qi21_weights(*([fake] * 15))
+    assert B.qi21_img_in_tokens(cfg, w, fake, 0, fake, 0) == B.QI21_ERR_INVALID_ARG
+    assert B.qi21_img_in_tokens(cfg, w, fake + 4, 4, fake, 0) == B.QI21_ERR_INVALID_ARG
