@@ -110,11 +110,22 @@ typedef struct {
  * qi21_prefix_extract; rows [P, P+N) are rewritten by every cached step with
  * that step's target K/V. state: QI21_CACHE_EMPTY until an extract succeeds. */
 enum { QI21_CACHE_EMPTY = 0, QI21_CACHE_EXTRACTED = 1 };
+
+/* Shared-prefix layout (denoise batching: several requests with the same text
+ * and reference images, [LAB] 6A "prefix K/V computed once, used by every
+ * step"): one prefix for all `batch` target requests. Per layer
+ * [2 (K,V)][Pp + batch*N][d], Pp = P rounded up to QI21_ATTN_KEY_TILE: rows
+ * [0, P) hold the prefix K/V written by one extract (prefix_hidden [1][P][d]),
+ * rows [P, Pp) are never read, and rows [Pp + b*N, Pp + (b+1)*N) hold request
+ * b's target K/V of the current step. Every request's attention reads the one
+ * copy of the prefix rows. Built by qi21_kv_cache_init_shared. */
+#define QI21_ATTN_KEY_TILE 128
 typedef struct {
     void *base;
     int32_t batch, n_prefix, n_target;
     int32_t n_layers, d_model, dtype;
     int32_t state;
+    int32_t shared_prefix;   /* 0: [L][2][B][P+N][d]; 1: the shared-prefix layout above */
 } qi21_kv_cache;
 
 /* ---------------------------------------------------------------- host helpers */
@@ -181,6 +192,10 @@ size_t qi21_workspace_bytes(const qi21_config *cfg, int32_t batch, int32_t n_pre
 /* Initialise a cache descriptor over caller memory (state EMPTY). */
 qi21_status qi21_kv_cache_init(qi21_kv_cache *cache, void *base, const qi21_config *cfg,
                                int32_t batch, int32_t n_prefix, int32_t n_target);
+/* The shared-prefix layout: bytes, and a descriptor (shared_prefix = 1). */
+size_t qi21_kv_cache_bytes_shared(const qi21_config *cfg, int32_t batch, int32_t n_prefix, int32_t n_target);
+qi21_status qi21_kv_cache_init_shared(qi21_kv_cache *cache, void *base, const qi21_config *cfg,
+                                      int32_t batch, int32_t n_prefix, int32_t n_target);
 
 /* ---------------------------------------------------------------- device entry points */
 

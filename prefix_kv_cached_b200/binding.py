@@ -52,7 +52,7 @@ class qi21_weights(ct.Structure):
 class qi21_kv_cache(ct.Structure):
     _fields_ = [("base", ct.c_void_p), ("batch", ct.c_int32), ("n_prefix", ct.c_int32),
                 ("n_target", ct.c_int32), ("n_layers", ct.c_int32), ("d_model", ct.c_int32),
-                ("dtype", ct.c_int32), ("state", ct.c_int32)]
+                ("dtype", ct.c_int32), ("state", ct.c_int32), ("shared_prefix", ct.c_int32)]
 
 
 class qi21_kernel_time(ct.Structure):
@@ -70,6 +70,9 @@ _SIGS = {
     "qi21_kv_cache_bytes": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
     "qi21_workspace_bytes": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
     "qi21_kv_cache_init": (_I32, [ct.POINTER(qi21_kv_cache), _P, ct.POINTER(qi21_config), _I32, _I32, _I32]),
+    "qi21_kv_cache_bytes_shared": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
+    "qi21_kv_cache_init_shared": (_I32, [ct.POINTER(qi21_kv_cache), _P, ct.POINTER(qi21_config), _I32, _I32,
+                                         _I32]),
     "qi21_modulation": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P, _P,
                                ct.c_size_t, _P]),
     "qi21_modulation_noalloc": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P,
@@ -194,6 +197,17 @@ def qi21_kv_cache_init(base, cfg, batch, n_prefix, n_target):
     cache = qi21_kv_cache()
     check("qi21_kv_cache_init", lib.qi21_kv_cache_init(ct.byref(cache), _addr(base), ct.byref(cfg), batch,
                                                        n_prefix, n_target))
+    return cache
+
+
+def qi21_kv_cache_bytes_shared(cfg, batch, n_prefix, n_target):
+    return lib.qi21_kv_cache_bytes_shared(ct.byref(cfg), batch, n_prefix, n_target)
+
+
+def qi21_kv_cache_init_shared(base, cfg, batch, n_prefix, n_target):
+    cache = qi21_kv_cache()
+    check("qi21_kv_cache_init_shared", lib.qi21_kv_cache_init_shared(ct.byref(cache), _addr(base), ct.byref(cfg),
+                                                                     batch, n_prefix, n_target))
     return cache
 
 

@@ -234,6 +234,10 @@ struct StackArgs {
     int kv_len;               // keys visible (rows of the K/V buffer per item)
     const int *kv_limit;      // [M] or null
     bool kv_only_last;        // extract: the last layer only needs K/V
+    // shared-prefix cache: the prefix rows [0, P) are one copy read by every item;
+    // item b's target rows start at Pp + b*N (kv_bstride = N*d, row_off = Pp)
+    bool shared;
+    int shared_P, shared_Pp;
 };
 
 template <typename T>
@@ -291,8 +295,14 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
         const uint64_t nl = a.kv_layer_stride ? (uint64_t)c.n_layers : 1;
         const uint64_t lstride = a.kv_layer_stride ? (uint64_t)a.kv_layer_stride : (uint64_t)a.kv_bstride * a.B;
         bool ok = make_map4(&maps.q4, a.q, d, R, 1, 1, d, (uint64_t)R * d, (uint64_t)R * d);
-        ok &= make_map4(&maps.k4, a.kv_k0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
-        ok &= make_map4(&maps.v4, a.kv_v0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
+        if (a.shared) {   // one item of Pp + B*N rows per layer
+            const uint64_t rows_all = (uint64_t)a.shared_Pp + (uint64_t)a.B * a.N;
+            ok &= make_map4(&maps.k4, a.kv_k0, d, rows_all, 1, nl, d, rows_all * d, lstride);
+            ok &= make_map4(&maps.v4, a.kv_v0, d, rows_all, 1, nl, d, rows_all * d, lstride);
+        } else {
+            ok &= make_map4(&maps.k4, a.kv_k0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
+            ok &= make_map4(&maps.v4, a.kv_v0, d, a.kv_len, a.B, nl, d, a.kv_bstride, lstride);
+        }
         ok &= make_map_f32(&maps.h32, a.h, d, R);
         if (!ok) {
             L.status = QI21_ERR_CUDA;
@@ -362,6 +372,12 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             ap.scale_log2 = 1.4426950408889634f / sqrtf((float)Dh);
             ap.layer = a.kv_layer_stride ? l : 0;
             ap.err = a.err;
+            if (a.shared) {
+                ap.shared_tiles = a.shared_Pp / QI21_ATTN_KEY_TILE;
+                ap.prefix_len = a.shared_P;
+                ap.tgt_len = a.N;
+                ap.tgt_row0 = a.shared_Pp;
+            }
             if (Dh == 128)
                 launch_attn_tc<128>(L, maps.q4, maps.k4, maps.v4, ap, a.B);
             else
@@ -375,8 +391,13 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             }
             dim3 grid((a.M + 31) / 32, H, a.B);
             L.run("attn_simt", [&] {
-                k_attn_simt<T><<<grid, 128, smem, L.st>>>(q, (int64_t)a.M * d, a.M, d, kdst, vdst, a.kv_bstride, d,
-                                                         a.kv_len, a.kv_limit, o, Dh, scale);
+                if (a.shared)
+                    k_attn_simt<T><<<grid, 128, smem, L.st>>>(q, (int64_t)a.M * d, a.M, d, kdst, vdst, 0, d, a.kv_len,
+                                                             a.kv_limit, o, Dh, scale, a.shared_P,
+                                                             (int64_t)a.shared_Pp * d, a.kv_bstride);
+                else
+                    k_attn_simt<T><<<grid, 128, smem, L.st>>>(q, (int64_t)a.M * d, a.M, d, kdst, vdst, a.kv_bstride, d,
+                                                             a.kv_len, a.kv_limit, o, Dh, scale, a.kv_len, 0, 0);
             });
         }
         if (tc) {
@@ -487,6 +508,12 @@ static qi21_status check_shapes(const qi21_config *c) {
 
 static qi21_status finish(Launcher &L) { return L.status; }
 
+// Shared-prefix cache: prefix rows padded to the attention key tile, then batch*N target rows.
+static int64_t padded_prefix_rows(int P) {
+    return ((int64_t)P + QI21_ATTN_KEY_TILE - 1) / QI21_ATTN_KEY_TILE * QI21_ATTN_KEY_TILE;
+}
+static int64_t shared_rows(int P, int N, int B) { return padded_prefix_rows(P) + (int64_t)B * N; }
+
 }  // namespace qi21
 
 using namespace qi21;
@@ -565,9 +592,11 @@ extern "C" qi21_status qi21_prefix_extract(const qi21_config *c, const qi21_weig
     if (!al16(prefix_hidden) || !al16(cos_sin_prefix) || !al16(kv_limit_prefix) || !al16(mod_row_prefix) ||
         !al16(ws))
         return QI21_ERR_INVALID_ARG;
-    const int B = cache->batch, P = cache->n_prefix, N = cache->n_target;
-    if (cache->n_layers != c->n_layers || cache->d_model != c->d_model || cache->dtype != c->dtype || B <= 0 ||
-        P <= 0 || N <= 0)
+    const int P = cache->n_prefix, N = cache->n_target;
+    const bool shared = cache->shared_prefix != 0;
+    const int B = shared ? 1 : cache->batch;          // a shared prefix is extracted once
+    if (cache->n_layers != c->n_layers || cache->d_model != c->d_model || cache->dtype != c->dtype ||
+        cache->batch <= 0 || P <= 0 || N <= 0)
         return QI21_ERR_CACHE_STATE;
     const WsLayout lay = ws_layout(*c, B, P, N);
     if (ws_bytes < lay.total) return QI21_ERR_WORKSPACE_TOO_SMALL;
@@ -584,7 +613,8 @@ extern "C" qi21_status qi21_prefix_extract(const qi21_config *c, const qi21_weig
     a.gemm = (float *)(wsb + lay.gemm); a.gates = (float *)(wsb + lay.gates); a.err = (uint32_t *)(wsb + lay.err);
     a.mod_lo = mod_row_prefix; a.mod_hi = mod_row_prefix;
     a.cos_sin = cos_sin_prefix;
-    const int64_t rows = (int64_t)P + N;
+    // rows per (layer, K|V) block: one item of Pp + batch*N rows (shared), else batch items of P + N rows
+    const int64_t rows = shared ? shared_rows(P, N, cache->batch) : (int64_t)P + N;
     a.kv_k0 = (char *)cache->base;
     a.kv_v0 = (char *)cache->base + eb * (size_t)B * rows * d;
     a.kv_layer_stride = 2 * (int64_t)B * rows * d;
@@ -619,6 +649,7 @@ extern "C" qi21_status qi21_cached_step(const qi21_config *c, const qi21_weights
         cache->dtype != c->dtype)
         return QI21_ERR_CACHE_STATE;
     const int B = cache->batch, P = cache->n_prefix, N = cache->n_target;
+    const bool shared = cache->shared_prefix != 0;
     const WsLayout lay = ws_layout(*c, B, P, N);
     if (ws_bytes < lay.total) return QI21_ERR_WORKSPACE_TOO_SMALL;
     char *wsb = (char *)ws;
@@ -633,13 +664,26 @@ extern "C" qi21_status qi21_cached_step(const qi21_config *c, const qi21_weights
     a.gemm = (float *)(wsb + lay.gemm); a.gates = (float *)(wsb + lay.gates); a.err = (uint32_t *)(wsb + lay.err);
     a.mod_lo = mod_row_target; a.mod_hi = mod_row_target;
     a.cos_sin = cos_sin_target;
-    const int64_t rows = (int64_t)P + N;
-    a.kv_k0 = (char *)cache->base;
-    a.kv_v0 = (char *)cache->base + eb * (size_t)B * rows * d;
-    a.kv_layer_stride = 2 * (int64_t)B * rows * d;
-    a.kv_bstride = rows * d;
-    a.row_off = P;
-    a.kv_len = (int)rows;
+    if (shared) {
+        const int64_t rows_all = shared_rows(P, N, B);
+        a.kv_k0 = (char *)cache->base;
+        a.kv_v0 = (char *)cache->base + eb * (size_t)rows_all * d;
+        a.kv_layer_stride = 2 * rows_all * d;
+        a.kv_bstride = (int64_t)N * d;            // item b's target rows start at Pp + b*N
+        a.row_off = (int)padded_prefix_rows(P);
+        a.kv_len = P + N;                         // keys each target row sees
+        a.shared = true;
+        a.shared_P = P;
+        a.shared_Pp = (int)padded_prefix_rows(P);
+    } else {
+        const int64_t rows = (int64_t)P + N;
+        a.kv_k0 = (char *)cache->base;
+        a.kv_v0 = (char *)cache->base + eb * (size_t)B * rows * d;
+        a.kv_layer_stride = 2 * (int64_t)B * rows * d;
+        a.kv_bstride = rows * d;
+        a.row_off = P;
+        a.kv_len = (int)rows;
+    }
     a.kv_limit = nullptr;
     a.kv_only_last = false;
     if (c->dtype == QI21_DTYPE_BF16) {

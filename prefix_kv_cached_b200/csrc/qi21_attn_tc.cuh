@@ -49,6 +49,11 @@ struct AttnParams {
     float scale_log2;     // log2(e) / sqrt(Dh)
     int layer;            // 4th coordinate of the K/V tensor maps
     uint32_t *err;
+    // Shared-prefix cache (one prefix for every item): key tiles [0, shared_tiles)
+    // are prefix rows t*BK (keys >= prefix_len masked), the rest item b's target
+    // rows tgt_row0 + b*tgt_len + (t - shared_tiles)*BK (keys >= tgt_len masked).
+    // shared_tiles == 0: every item's keys are rows [0, kv_len) of its own block.
+    int shared_tiles, prefix_len, tgt_len, tgt_row0;
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -88,6 +93,8 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *m, 
 
 // Named barrier over the 256 softmax threads (id 1; id 0 is __syncthreads).
 __device__ __forceinline__ void softmax_bar_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+static_assert(QI21_ATTN_KEY_TILE == 128, "the shared-prefix padding is the attention key tile");
 
 template <int DH>
 struct AttnCfg {
@@ -182,8 +189,15 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     const uint32_t tmem_base = *tmem_slot;
     const int kv_end = *kv_end_s;
-    const int T = (kv_end + C::BK - 1) / C::BK;
+    const int T = p.shared_tiles > 0 ? p.shared_tiles + (p.tgt_len + C::BK - 1) / C::BK
+                                     : (kv_end + C::BK - 1) / C::BK;
     const int TA = (T + 1) >> 1, TB = T >> 1;     // tiles of half A and half B
+    // row and item coordinates of key tile t in the K/V tensor maps
+    auto tile_row = [&](int t) -> int {
+        if (p.shared_tiles == 0) return t * C::BK;
+        return t < p.shared_tiles ? t * C::BK : p.tgt_row0 + b * p.tgt_len + (t - p.shared_tiles) * C::BK;
+    };
+    const int kv_item = p.shared_tiles > 0 ? 0 : b;
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producers
@@ -201,7 +215,7 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_arrive_expect_tx(kb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
                     tma_load_4d(smem_u32(smem + C::OFF_K + s * C::KV_BYTES + x * (C::BK * 128)), &tmK, kb,
-                                hh * DH + x * 64, tile * C::BK, b, p.layer);
+                                hh * DH + x * 64, tile_row(tile), kv_item, p.layer);
             }
         } else if (lane == 1 && T > 0) {
             for (int n = 0; n < T; ++n) {
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(320, 1)
                 mbar_arrive_expect_tx(vb, C::KV_BYTES);
                 for (int x = 0; x < C::BOXES; ++x)
                     tma_load_4d(smem_u32(smem + C::OFF_V + s * C::KV_BYTES + x * (C::BK * 128)), &tmV, vb,
-                                hh * DH + x * 64, tile * C::BK, b, p.layer);
+                                hh * DH + x * 64, tile_row(tile), kv_item, p.layer);
             }
         }
     } else if (warp == 1) {
@@ -313,11 +327,21 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) tmem_ld32(t_s + cc * 32, sv[cc]);
             tmem_wait_ld();
-            const int key0 = (tile0 + j) * C::BK;
-            if (key0 + C::BK > lim) {
+            // keys of this tile and the first masked one
+            const int t = tile0 + j;
+            int key0 = t * C::BK, klim = lim;
+            if (p.shared_tiles > 0) {
+                if (t < p.shared_tiles) {
+                    klim = min(lim, p.prefix_len);
+                } else {
+                    key0 = (t - p.shared_tiles) * C::BK;
+                    klim = p.tgt_len;
+                }
+            }
+            if (key0 + C::BK > klim) {
 #pragma unroll
                 for (int i = 0; i < 128; ++i)
-                    if (key0 + i >= lim) sv[i >> 5][i & 31] = -INFINITY;
+                    if (key0 + i >= klim) sv[i >> 5][i & 31] = -INFINITY;
             }
             float m8[8];
 #pragma unroll

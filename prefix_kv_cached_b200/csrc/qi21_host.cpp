@@ -193,6 +193,16 @@ extern "C" size_t qi21_kv_cache_bytes(const qi21_config *c, int32_t B, int32_t P
            (size_t)c->d_model;
 }
 
+static int64_t padded_prefix(int32_t P) {
+    return ((int64_t)P + QI21_ATTN_KEY_TILE - 1) / QI21_ATTN_KEY_TILE * QI21_ATTN_KEY_TILE;
+}
+
+extern "C" size_t qi21_kv_cache_bytes_shared(const qi21_config *c, int32_t B, int32_t P, int32_t N) {
+    if (!qi21_config_ok(c) || B <= 0 || P <= 0 || N <= 0) return 0;
+    return qi21::dtype_bytes(c->dtype) * (size_t)c->n_layers * 2 * (size_t)(padded_prefix(P) + (int64_t)B * N) *
+           (size_t)c->d_model;
+}
+
 extern "C" size_t qi21_workspace_bytes(const qi21_config *c, int32_t B, int32_t P, int32_t N) {
     if (!qi21_config_ok(c) || B <= 0 || P < 0 || N <= 0) return 0;
     return qi21::ws_layout(*c, B, P, N).total;
@@ -211,5 +221,13 @@ extern "C" qi21_status qi21_kv_cache_init(qi21_kv_cache *cache, void *base, cons
     cache->d_model = c->d_model;
     cache->dtype = c->dtype;
     cache->state = QI21_CACHE_EMPTY;
+    cache->shared_prefix = 0;
     return QI21_OK;
+}
+
+extern "C" qi21_status qi21_kv_cache_init_shared(qi21_kv_cache *cache, void *base, const qi21_config *c,
+                                                 int32_t B, int32_t P, int32_t N) {
+    qi21_status s = qi21_kv_cache_init(cache, base, c, B, P, N);
+    if (s == QI21_OK) cache->shared_prefix = 1;
+    return s;
 }

@@ -352,7 +352,10 @@ __global__ void __launch_bounds__(128) k_attn_simt(const T *__restrict__ q, int6
                                                    const T *__restrict__ kb, const T *__restrict__ vb,
                                                    int64_t kv_bstride, int ldkv, int kv_len,
                                                    const int *__restrict__ kv_limit, T *__restrict__ out, int Dh,
-                                                   float scale) {
+                                                   float scale, int split, int64_t tgt_off, int64_t tgt_bstride) {
+    // keys [0, split) are rows of kb + b*kv_bstride; keys k >= split are rows
+    // k - split of kb + tgt_off + b*tgt_bstride (the shared-prefix cache; split =
+    // kv_len otherwise)
     extern __shared__ float sm[];
     const int DP = Dh + 1;
     float *Qs = sm;                 // [32][DP]
@@ -389,9 +392,13 @@ __global__ void __launch_bounds__(128) k_attn_simt(const T *__restrict__ q, int6
         __syncthreads();
         for (int e = tid; e < 32 * Dh; e += 128) {
             const int i = e / Dh, j = e % Dh;
-            const bool ok = t0 + i < kv_len;
-            Ks[i * DP + j] = ok ? to_f(kbb[(size_t)(t0 + i) * ldkv + j]) : 0.f;
-            Vs[i * DP + j] = ok ? to_f(vbb[(size_t)(t0 + i) * ldkv + j]) : 0.f;
+            const int key = t0 + i;
+            const bool ok = key < kv_len;
+            const size_t off = key < split ? (size_t)key * ldkv : (size_t)(tgt_off - (int64_t)b * kv_bstride) +
+                                                                     (size_t)b * tgt_bstride +
+                                                                     (size_t)(key - split) * ldkv;
+            Ks[i * DP + j] = ok ? to_f(kbb[off + j]) : 0.f;
+            Vs[i * DP + j] = ok ? to_f(vbb[off + j]) : 0.f;
         }
         __syncthreads();
         float s[8];

@@ -33,7 +33,11 @@ def lab_rope_omega(base: float = 10000.0) -> np.ndarray:
 
 class Qi21Runner:
     def __init__(self, workload: C.Workload, dtype: int = B.QI21_DTYPE_F32, device: str = "cuda",
-                 host_weights: Optional[Dict[str, np.ndarray]] = None, frame_mode: int = 0):
+                 host_weights: Optional[Dict[str, np.ndarray]] = None, frame_mode: int = 0,
+                 shared_prefix: bool = False, share_weights_with: Optional["Qi21Runner"] = None):
+        """shared_prefix: the batch items are requests sharing one prefix (one
+        extract from prefix_hidden [1][P][d], every request's attention reading
+        the one copy); share_weights_with: reuse another runner's device weights."""
         self.w = workload
         self.shape = workload.shape
         self.dtype = dtype
@@ -54,7 +58,11 @@ class Qi21Runner:
         self.kv_limit_all = lim
         self.kv_limit_prefix = lim[: self.P].contiguous()
         self.weights: Dict[str, torch.Tensor] = {}
+        self.shared_prefix = shared_prefix
         for name, shp in C.weight_specs(sh):
+            if share_weights_with is not None:
+                self.weights[name] = share_weights_with.weights[name]
+                continue
             sdt = torch.float32 if name in ("q_norm", "k_norm") else self.tdtype
             if host_weights is not None:
                 self.weights[name] = torch.from_numpy(np.ascontiguousarray(host_weights[name])).to(
@@ -64,9 +72,14 @@ class Qi21Runner:
         self.wstruct = B.qi21_weights(*[self.weights[n].data_ptr() for n in (
             "w_img_in", "w_out", "w_t1", "w_t2", "w_mod", "w_fin", "w_q", "w_k", "w_v", "w_o", "w_gate", "w_up",
             "w_down", "q_norm", "k_norm")])
-        kvb = B.qi21_kv_cache_bytes(self.cfg, self.Bn, self.P, self.N)
-        self.cache_buf = torch.zeros(kvb, dtype=torch.uint8, device=self.device)
-        self.cache = B.qi21_kv_cache_init(self.cache_buf, self.cfg, self.Bn, self.P, self.N)
+        if shared_prefix:
+            kvb = B.qi21_kv_cache_bytes_shared(self.cfg, self.Bn, self.P, self.N)
+            self.cache_buf = torch.zeros(kvb, dtype=torch.uint8, device=self.device)
+            self.cache = B.qi21_kv_cache_init_shared(self.cache_buf, self.cfg, self.Bn, self.P, self.N)
+        else:
+            kvb = B.qi21_kv_cache_bytes(self.cfg, self.Bn, self.P, self.N)
+            self.cache_buf = torch.zeros(kvb, dtype=torch.uint8, device=self.device)
+            self.cache = B.qi21_kv_cache_init(self.cache_buf, self.cfg, self.Bn, self.P, self.N)
         self.ws_bytes = B.qi21_workspace_bytes(self.cfg, self.Bn, self.P, self.N)
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.device)
         nch = sh.n_chunks
@@ -160,8 +173,14 @@ class Qi21Runner:
         B.check("qi21_check_device_error", B.qi21_check_device_error(self.ws, self.ws_bytes, self.stream))
 
     def cache_kv(self):
-        """Views of the cache as K, V [L][B][P+N][H][Dh] (for tests)."""
+        """Views of the cache as K, V [L][B][P+N][H][Dh] (for tests); with a shared
+        prefix, [L][Pp + B*N][H][Dh] (prefix rows [0, P), request b at Pp + b*N)."""
         sh = self.shape
+        if self.shared_prefix:
+            pp = -(-self.P // 128) * 128
+            t = self.cache_buf.view(self.tdtype).view(sh.n_layers, 2, pp + self.Bn * self.N, sh.n_heads,
+                                                      sh.head_dim)
+            return t[:, 0], t[:, 1]
         t = self.cache_buf.view(self.tdtype).view(sh.n_layers, 2, self.Bn, self.P + self.N, sh.n_heads,
                                                   sh.head_dim)
         return t[:, 0], t[:, 1]

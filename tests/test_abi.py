@@ -195,3 +195,19 @@ def test_packing_errors_and_validation(B):
     w = B.qi21_weights(*([fake] * 15))
     assert B.qi21_img_in_tokens(cfg, w, fake, 0, fake, 0) == B.QI21_ERR_INVALID_ARG
     assert B.qi21_img_in_tokens(cfg, w, fake + 4, 4, fake, 0) == B.QI21_ERR_INVALID_ARG
+
+
+def test_shared_prefix_cache_layout(B):
+    cfg = _cfg(B)
+    fake = 0x10000
+    # [L][2][Pp + B*N][d], Pp = P rounded up to the 128-key attention tile
+    for P, N, Bn in ((8, 4, 3), (128, 4, 1), (129, 7, 2)):
+        pp = -(-P // 128) * 128
+        assert B.qi21_kv_cache_bytes_shared(cfg, Bn, P, N) == 4 * cfg.n_layers * 2 * (pp + Bn * N) * cfg.d_model
+    cache = B.qi21_kv_cache_init_shared(fake, cfg, 3, 8, 4)
+    assert (cache.shared_prefix, cache.batch, cache.state) == (1, 3, B.QI21_CACHE_EMPTY)
+    assert B.qi21_kv_cache_init(fake, cfg, 3, 8, 4).shared_prefix == 0
+    ws_bytes = B.qi21_workspace_bytes(cfg, 3, 8, 4)
+    w = B.qi21_weights(*([fake] * 15))
+    assert B.qi21_cached_step(cfg, w, cache, fake, fake, fake, fake, fake, fake, ws_bytes, 0) == \
+        B.QI21_ERR_CACHE_STATE
