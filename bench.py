@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-image CUDA-graph timing")
+    ap.add_argument("--batched-requests", type=int, default=4,
+                    help="requests sharing one prefix cache in the denoise-batching timing (0: skip)")
     return ap.parse_args()
 
 
@@ -428,6 +430,43 @@ def main():
                  "then per step modulation from the device sigma table, cached step, Euler"}
         del graph
 
+    # denoise batching: several requests sharing one prefix cache (one extract; every
+    # request's attention reads the single copy of the prefix K/V), stepped together
+    batched = None
+    if args.batched_requests > 1:
+        import dataclasses
+        from qi21_synth.gen import normal_torch as _nt
+        wr = dataclasses.replace(w, batch=args.batched_requests)
+        rb = Qi21Runner(wr, B.QI21_DTYPE_BF16, device=str(dev), shared_prefix=True, share_weights_with=r)
+        xb = _nt(seed_w.seed + 1, "noise", (wr.batch, w.n_target, sh.latent_ch), device=dev, dtype=torch.float32)
+        vb = torch.empty_like(xb)
+        rb.set_prefix_row()
+        rb.prefix_extract(pre[:1].contiguous())
+
+        def bstep(k):
+            i = k % (len(sig) - 1)
+            rb.set_target_row(sig[i]); rb.cached_step(xb, vb); rb.euler(xb, vb, sig[i], sig[i + 1], xb)
+
+        for k in range(2):
+            bstep(k)
+        torch.cuda.synchronize()
+        rb.check_device()
+        nb = max(4, args.steps // 2)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist_barrier(world)
+        torch.cuda.synchronize()
+        c0.record(st)
+        for k in range(nb):
+            bstep(k)
+        c1.record(st)
+        torch.cuda.synchronize()
+        rb.check_device()
+        b_ms = dist_max(c0.elapsed_time(c1), world) / nb
+        batched = {"requests": wr.batch, "ms_per_step": round(b_ms, 3), "steps": nb,
+                   "target_tokens_per_s": round(world * wr.batch * w.n_target / (b_ms / 1e3), 1),
+                   "how": "one shared prefix cache (extracted once), all requests' target tokens in each step"}
+        del rb, xb, vb
+
     # e2e: same step through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None
     if not args.no_e2e:
@@ -492,6 +531,7 @@ def main():
             "tensor_frac_step": round(step_tflops / peaks["bf16_tflops_sustained"], 4),
             "step_tflops": round(step_tflops, 1),
             "step_ms_percentiles": pct,
+            "batched_shared_prefix": batched,
             "per_image": {"extract_ms": round(extract_ms, 3),
                           "tokens_per_s": round(world * tokens / ((extract_ms + 8 * ms_step) / 1e3), 1),
                           "graph": image},
