@@ -41,6 +41,7 @@ struct GemmParams {
     int m_blocks;      // ceil(R / 128)
     int n_blocks;      // output tiles along N
     int ksplit;        // EPI_RESIDUAL: K slices per output tile, each reduce-added into h (1 otherwise)
+    int group_m;       // row blocks per band of the tile order (0: all of them)
     int M, split;      // rows per item; rows m < split read the prefix modulation row
     // EPI_RESIDUAL
     float *h;
@@ -100,10 +101,19 @@ __device__ __forceinline__ void store_bf16x32(bf16 *dst, const float (&v)[32]) {
 // partial product is reduce-added into h like a whole tile's.
 __device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int kblocks, int &m_blk, int &n_blk,
                                             int &kb0, int &kb1) {
-    m_blk = tile % p.m_blocks;
-    const int rest = tile / p.m_blocks;
-    n_blk = rest % p.n_blocks;
-    const int ks = rest / p.n_blocks;
+    // K slice outermost; inside a slice, bands of group_m row blocks, and inside a
+    // band the row block varies fastest, so the CTAs running together read a band
+    // of A rows and a run of B rows instead of all of A.
+    const int per_slice = p.m_blocks * p.n_blocks;
+    const int ks = tile / per_slice;
+    const int t = tile - ks * per_slice;
+    const int gm = p.group_m > 0 ? p.group_m : p.m_blocks;
+    const int band = t / (gm * p.n_blocks);
+    const int m0 = band * gm;
+    const int rows = min(gm, p.m_blocks - m0);
+    const int local = t - band * gm * p.n_blocks;
+    m_blk = m0 + local % rows;
+    n_blk = local / rows;
     kb0 = (int)((int64_t)kblocks * ks / p.ksplit);
     kb1 = (int)((int64_t)kblocks * (ks + 1) / p.ksplit);
 }
