@@ -30,7 +30,10 @@
 // of one issuing thread execute in issue order, so that PV reads P_X before the
 // next S_X overwrites it. A commit tracks every earlier MMA of the thread, so
 // when S_X(j) is complete, PV_X(j-1) is too: the softmax may then rescale O_X
-// and write P_X(j) without a further wait.
+// and write P_X(j) without a further wait. The softmax signals P_X(j) in two
+// parts (keys 0..63, then 64..127; any O rescale before the first), and the MMA
+// warp issues the first half of PV_X(j) on the first signal, so it runs while
+// the second half of the exponentials is computed.
 // The running max of a row moves only when a tile raises it by more than 2^8
 // (exp2 domain); otherwise P = exp2(S c - m c) <= 256 is formed against the
 // stale max, which the final 1/l normalisation absorbs.
@@ -142,8 +145,8 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t *v_full = k_empty + C::SK;   // [SV]
     uint64_t *v_empty = v_full + C::SV;   // [SV] (the PV MMA reading that stage is done)
     uint64_t *s_full = v_empty + C::SV;   // [2 halves]
-    uint64_t *p_full = s_full + 2;        // [2 halves] (softmax wrote P and finished with O)
-    uint64_t *o_full = p_full + 2;        // every MMA done
+    uint64_t *p_full = s_full + 2;        // [half][part]: softmax wrote P (keys 64*part ..) and finished with O
+    uint64_t *o_full = p_full + 4;        // every MMA done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 1);
     static_assert((1 + 2 * C::SK + 2 * C::SV + 5) * 8 + 16 <= 256, "barrier region");
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -165,7 +168,8 @@ __global__ void __launch_bounds__(320, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_full[i]), 1);
-            mbar_init(smem_u32(&p_full[i]), C::HALF_THREADS);
+            mbar_init(smem_u32(&p_full[2 * i]), C::HALF_THREADS);
+            mbar_init(smem_u32(&p_full[2 * i + 1]), C::HALF_THREADS);
         }
         mbar_init(smem_u32(o_full), 1);
         *abort_flag = 0;
@@ -267,16 +271,28 @@ __global__ void __launch_bounds__(320, 1)
                 return true;
             };
             auto issue_pv = [&](int h, int j) -> bool {
-                if (!wait_warp(&p_full[h], j & 1)) return false;
+                if (!wait_warp(&p_full[2 * h], j & 1)) return false;
                 const int s = nv % C::SV;
                 if (!wait_warp(&v_full[s], (nv / C::SV) & 1)) return false;
                 tc_fence_after();
+                // keys 0..63 of P as soon as they are written, keys 64..127 after the
+                // second signal: the first half of PV runs under the rest of the softmax
+                const uint64_t dv = dv0 + s * KV_UNITS;
+                constexpr int KSTEPS = C::BK / 16;
                 if (leader) {
-                    const uint64_t dv = dv0 + s * KV_UNITS;
 #pragma unroll
-                    for (int k = 0; k < C::BK / 16; ++k)
+                    for (int k = 0; k < KSTEPS / 2; ++k)
                         umma_f16_ts(tmem_base + 256 + h * DH, tmem_base + h * 128 + k * 8, dv + k * 128, idesc_o,
                                     (j > 0 || k > 0) ? 1u : 0u);
+                }
+                __syncwarp();
+                if (!wait_warp(&p_full[2 * h + 1], j & 1)) return false;
+                tc_fence_after();
+                if (leader) {
+#pragma unroll
+                    for (int k = KSTEPS / 2; k < KSTEPS; ++k)
+                        umma_f16_ts(tmem_base + 256 + h * DH, tmem_base + h * 128 + k * 8, dv + k * 128, idesc_o,
+                                    1u);
                     umma_commit(smem_u32(&v_empty[s]));
                 }
                 __syncwarp();
@@ -362,6 +378,12 @@ __global__ void __launch_bounds__(320, 1)
             float s8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) s8[i] = 0.f;
+            // P ready for the PV MMA, in two parts: keys 0..63, then 64..127
+            auto signal_p = [&](int part) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&p_full[2 * h + part]));
+            };
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t u[16];
@@ -383,27 +405,27 @@ __global__ void __launch_bounds__(320, 1)
                     u[q] = pack_bf16x2(e[0], e[1]);
                 }
                 tmem_st16(t_s + cc * 16, u);               // P_h: keys 32cc .. 32cc+31
-            }
-            if (__any_sync(0xffffffffu, grow && !first)) {
-                // O_h holds PV_h(0..j-1) against the old max (complete: S_h(j) was
-                // issued after PV_h(j-1)); alpha = 1 on rows whose max did not move.
-                // Done after P so that the S registers are free.
-                float ov[32];
+                if (cc == 1) {
+                    // O rescale (rare) before the first P signal, so that PV_h(j) sees the
+                    // rescaled O. O_h holds PV_h(0..j-1) against the old max (complete: S_h(j)
+                    // was issued after PV_h(j-1)); alpha = 1 on rows whose max did not move.
+                    if (__any_sync(0xffffffffu, grow && !first)) {
+                        float ov[32];
 #pragma unroll
-                for (int cc = 0; cc < DH / 32; ++cc) {
-                    tmem_ld32(t_o + cc * 32, ov);
-                    tmem_wait_ld();
-                    uint32_t u[32];
+                        for (int oc = 0; oc < DH / 32; ++oc) {
+                            tmem_ld32(t_o + oc * 32, ov);
+                            tmem_wait_ld();
+                            uint32_t w32[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(ov[i] * alpha);
-                    tmem_st32(t_o + cc * 32, u);
+                            for (int i = 0; i < 32; ++i) w32[i] = __float_as_uint(ov[i] * alpha);
+                            tmem_st32(t_o + oc * 32, w32);
+                        }
+                    }
+                    signal_p(0);
                 }
-                tmem_wait_st();
             }
-            tmem_wait_st();
+            signal_p(1);
             l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-            tc_fence_before();
-            mbar_arrive(smem_u32(&p_full[h]));
         }
         // merge the halves: each publishes its (m, l) per row; half h then writes
         // output columns [h Dh/2, (h+1) Dh/2) of its rows from O_A and O_B
