@@ -87,3 +87,37 @@ def test_full_width_cached_step_equals_recompute(B):
     a, b = v_c.double().cpu().numpy(), v_f.double().cpu().numpy()
     assert rel_l2(a, b) < BF16_TOL
     assert np.linalg.norm(a) > 0
+
+
+@pytest.mark.parametrize("name", ["mid", "block"])
+def test_f32_matches_oracle_at_benchmark_sizes(B, name):
+    """F32 storage (CUDA-core kernels) against the fp64 oracle at the benchmark's
+    block sizes: max relative error < 1e-4 on v_theta, the latent and the prefix K/V."""
+    from prefix_kv_cached_b200.runner import Qi21Runner
+    from tests._harness import max_rel
+    w = C.make_workload(name)
+    model, wts = oracle_model(w, "float32")
+    r = Qi21Runner(w, B.QI21_DTYPE_F32, host_weights=wts)
+    pre = C.host_prefix_hidden(w)
+    x0 = C.host_noise(w)
+    x = torch.from_numpy(x0.astype(np.float32)).cuda()
+    v = torch.empty_like(x)
+    r.set_prefix_row()
+    r.prefix_extract(torch.from_numpy(pre.astype(np.float32)).cuda())
+    r.set_target_row(w.sigmas[0])
+    r.cached_step(x, v)
+    r.euler(x, v, w.sigmas[0], w.sigmas[1], x)
+    torch.cuda.synchronize()
+    r.check_device()
+    K, V = r.cache_kv()
+    gv, gx = v.double().cpu().numpy(), x.double().cpu().numpy()
+    seq = O.make_sequence(w.segments)
+    m0, _ = O.modulation(0.0, model.wts, 4)
+    mt, sf = O.modulation(1000.0 * w.sigmas[0], model.wts, 4)
+    for b in ((0, w.batch - 1) if w.batch > 1 else (0,)):
+        ck, cv = O.prefix_extract(model, seq, pre[b], m0)
+        assert max_rel(K[:, b, :r.P].double().cpu().numpy(), ck) < 1e-4
+        assert max_rel(V[:, b, :r.P].double().cpu().numpy(), cv) < 1e-4
+        vo, _ = O.cached_step(model, seq, ck, cv, x0[b], mt, sf)
+        assert max_rel(gv[b], vo) < 1e-4
+        assert max_rel(gx[b], O.euler_step(x0[b], vo, w.sigmas[0], w.sigmas[1])) < 1e-4
