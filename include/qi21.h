@@ -102,6 +102,19 @@ typedef struct {
     const float *q_norm, *k_norm;
 } qi21_weights;
 
+/* The same weights as row-major [in][out] matrices (the lab's y = x @ W), device
+ * pointers in the config dtype, per-layer tensors stacked on a leading layer axis:
+ *   w_img_in [C][d], w_out [d][C], w_t1 [time_dim][d], w_t2 [d][d],
+ *   w_mod [d][chunks*d], w_fin [d][d], w_q/w_k/w_v/w_o [L][d][d],
+ *   w_gate/w_up [L][d][F], w_down [L][F][d]; q_norm, k_norm [L][head_dim] float32. */
+typedef struct {
+    const void *w_img_in, *w_out;
+    const void *w_t1, *w_t2, *w_mod, *w_fin;
+    const void *w_q, *w_k, *w_v, *w_o;
+    const void *w_gate, *w_up, *w_down;
+    const float *q_norm, *k_norm;
+} qi21_weights_canonical;
+
 /* Prefix K/V cache ([LAB] 6A; [E2E] §6 "kv_cache_mode"): one caller-owned
  * device buffer of qi21_kv_cache_bytes(), laid out [L][2 (K,V)][B][P+N][d]
  * in the config dtype. For layer l, item b, row r, head h, dim j the K value
@@ -182,6 +195,10 @@ qi21_status qi21_build_packing(const qi21_segment *segments, int32_t n_segments,
  * [cos(t f_i) ..., sin(t f_i) ...], f_i = 10000^(-2i/time_dim), t = 1000*sigma
  * ([LAB] 3B, [3B] §1). */
 qi21_status qi21_timestep_embedding(double t, int32_t time_dim, float *emb);
+
+/* Bytes of the packed weight buffer of qi21_pack_weights (every tensor in the
+ * [out][in] layout of qi21_weights, each starting on a 256-byte boundary). */
+size_t qi21_packed_weights_bytes(const qi21_config *cfg);
 
 /* Sizes in bytes of the caller-allocated buffers. */
 size_t qi21_kv_cache_bytes(const qi21_config *cfg, int32_t batch, int32_t n_prefix, int32_t n_target);
@@ -282,6 +299,15 @@ qi21_status qi21_full_recompute_step(const qi21_config *cfg, const qi21_weights 
  * x_out may alias x_k. */
 qi21_status qi21_euler_update(const float *x_k, const float *v, double sigma_k, double sigma_k1,
                               float *x_out, int64_t n, void *stream);
+
+/* Pack canonical [in][out] weights into the layout the kernels read: every
+ * matrix transposed to [out][in] (layer by layer for stacked tensors) into the
+ * caller's device buffer `packed` (qi21_packed_weights_bytes bytes, 256-byte
+ * aligned), the QK-norm vectors copied; *w receives pointers into `packed`.
+ * Data movement only: exact. Returns QI21_ERR_INVALID_ARG for null or
+ * misaligned pointers, QI21_ERR_WORKSPACE_TOO_SMALL if packed_bytes is short. */
+qi21_status qi21_pack_weights(const qi21_config *cfg, const qi21_weights_canonical *canonical,
+                              void *packed, size_t packed_bytes, qi21_weights *w, void *stream);
 
 /* Joint packing of the prefix values on the device ([2A] mechanisms (1)-(2);
  * [LAB] 2A). For item b and prefix token s:

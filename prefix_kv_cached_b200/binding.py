@@ -49,6 +49,12 @@ class qi21_weights(ct.Structure):
                                            "w_v", "w_o", "w_gate", "w_up", "w_down", "q_norm", "k_norm")]
 
 
+class qi21_weights_canonical(ct.Structure):
+    """Same fields as qi21_weights, row-major [in][out] matrices."""
+    _fields_ = [(n, ct.c_void_p) for n in ("w_img_in", "w_out", "w_t1", "w_t2", "w_mod", "w_fin", "w_q", "w_k",
+                                           "w_v", "w_o", "w_gate", "w_up", "w_down", "q_norm", "k_norm")]
+
+
 class qi21_kv_cache(ct.Structure):
     _fields_ = [("base", ct.c_void_p), ("batch", ct.c_int32), ("n_prefix", ct.c_int32),
                 ("n_target", ct.c_int32), ("n_layers", ct.c_int32), ("d_model", ct.c_int32),
@@ -70,6 +76,9 @@ _SIGS = {
     "qi21_kv_cache_bytes": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
     "qi21_workspace_bytes": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
     "qi21_kv_cache_init": (_I32, [ct.POINTER(qi21_kv_cache), _P, ct.POINTER(qi21_config), _I32, _I32, _I32]),
+    "qi21_packed_weights_bytes": (ct.c_size_t, [ct.POINTER(qi21_config)]),
+    "qi21_pack_weights": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights_canonical), _P, ct.c_size_t,
+                                 ct.POINTER(qi21_weights), _P]),
     "qi21_kv_cache_bytes_shared": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
     "qi21_kv_cache_init_shared": (_I32, [ct.POINTER(qi21_kv_cache), _P, ct.POINTER(qi21_config), _I32, _I32,
                                          _I32]),
@@ -198,6 +207,17 @@ def qi21_kv_cache_init(base, cfg, batch, n_prefix, n_target):
     check("qi21_kv_cache_init", lib.qi21_kv_cache_init(ct.byref(cache), _addr(base), ct.byref(cfg), batch,
                                                        n_prefix, n_target))
     return cache
+
+
+def qi21_packed_weights_bytes(cfg):
+    return lib.qi21_packed_weights_bytes(ct.byref(cfg))
+
+
+def qi21_pack_weights(cfg, canonical, packed, packed_bytes, stream=0):
+    """Returns (status, qi21_weights pointing into `packed`)."""
+    w = qi21_weights()
+    st = lib.qi21_pack_weights(ct.byref(cfg), ct.byref(canonical), _addr(packed), packed_bytes, ct.byref(w), stream)
+    return st, w
 
 
 def qi21_kv_cache_bytes_shared(cfg, batch, n_prefix, n_target):

@@ -768,6 +768,52 @@ extern "C" qi21_status qi21_euler_update(const float *x_k, const float *v, doubl
     return finish(L);
 }
 
+extern "C" qi21_status qi21_pack_weights(const qi21_config *c, const qi21_weights_canonical *cw, void *packed,
+                                         size_t packed_bytes, qi21_weights *w, void *stream) {
+    qi21_status s = check_shapes(c);
+    if (s) return s;
+    if (!cw || !w || !al16(packed)) return QI21_ERR_INVALID_ARG;
+    const void *src[15] = {cw->w_img_in, cw->w_out, cw->w_t1,   cw->w_t2,   cw->w_mod, cw->w_fin, cw->w_q,     cw->w_k,
+                           cw->w_v,      cw->w_o,   cw->w_gate, cw->w_up,   cw->w_down, cw->q_norm, cw->k_norm};
+    for (const void *p : src)
+        if (!al16(p)) return QI21_ERR_INVALID_ARG;
+    const PackedLayout lay = packed_layout(*c);
+    if (packed_bytes < lay.total) return QI21_ERR_WORKSPACE_TOO_SMALL;
+    const int d = c->d_model, C = c->latent_ch, T = c->time_dim, F = c->mlp_hidden, L = c->n_layers;
+    const int nch = c->use_shift ? 6 : 4;
+    // canonical [in][out] (rows = in, cols = out) per matrix, and how many are stacked
+    const int rows[13] = {C, d, T, d, d, d, d, d, d, d, d, d, F};
+    const int cols[13] = {d, C, d, d, nch * d, d, d, d, d, d, F, F, d};
+    const int nmat[13] = {1, 1, 1, 1, 1, 1, L, L, L, L, L, L, L};
+    char *base = (char *)packed;
+    void *dst[15];
+    for (int i = 0; i < 15; ++i) dst[i] = base + lay.off[i];
+    cudaStream_t st = (cudaStream_t)stream;
+    Launcher L_(st);
+    for (int i = 0; i < 13; ++i) {
+        dim3 grid((cols[i] + 31) / 32, (rows[i] + 31) / 32, nmat[i]);
+        if (c->dtype == QI21_DTYPE_BF16)
+            L_.run("transpose", [&] {
+                k_transpose<bf16><<<grid, 256, 0, st>>>((const bf16 *)src[i], (bf16 *)dst[i], rows[i], cols[i]);
+            });
+        else
+            L_.run("transpose", [&] {
+                k_transpose<float><<<grid, 256, 0, st>>>((const float *)src[i], (float *)dst[i], rows[i], cols[i]);
+            });
+    }
+    for (int i = 13; i < 15; ++i)
+        if (cudaMemcpyAsync(dst[i], src[i], sizeof(float) * (size_t)L * c->head_dim, cudaMemcpyDeviceToDevice, st) !=
+            cudaSuccess)
+            return QI21_ERR_CUDA;
+    const qi21_status fs = finish(L_);
+    if (fs) return fs;
+    w->w_img_in = dst[0]; w->w_out = dst[1]; w->w_t1 = dst[2]; w->w_t2 = dst[3]; w->w_mod = dst[4];
+    w->w_fin = dst[5]; w->w_q = dst[6]; w->w_k = dst[7]; w->w_v = dst[8]; w->w_o = dst[9];
+    w->w_gate = dst[10]; w->w_up = dst[11]; w->w_down = dst[12];
+    w->q_norm = (const float *)dst[13]; w->k_norm = (const float *)dst[14];
+    return QI21_OK;
+}
+
 extern "C" qi21_status qi21_pack_prefix(int32_t B, int32_t P, int32_t d, int32_t n_slots, int32_t n_img,
                                         const float *ctx, const float *img_tokens, const int32_t *slot_of,
                                         const int32_t *img_row, int32_t mode, float *out, void *stream) {

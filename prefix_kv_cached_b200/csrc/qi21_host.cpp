@@ -203,6 +203,11 @@ extern "C" size_t qi21_kv_cache_bytes_shared(const qi21_config *c, int32_t B, in
            (size_t)c->d_model;
 }
 
+extern "C" size_t qi21_packed_weights_bytes(const qi21_config *c) {
+    if (!qi21_config_ok(c)) return 0;
+    return qi21::packed_layout(*c).total;
+}
+
 extern "C" size_t qi21_workspace_bytes(const qi21_config *c, int32_t B, int32_t P, int32_t N) {
     if (!qi21_config_ok(c) || B <= 0 || P < 0 || N <= 0) return 0;
     return qi21::ws_layout(*c, B, P, N).total;

@@ -31,6 +31,29 @@ inline size_t dtype_bytes(int32_t dtype) { return dtype == QI21_DTYPE_BF16 ? 2 :
 // Kernel family of the BF16 mode (process-wide; qi21_set_tensor_cores).
 bool tc_enabled();
 
+// Packed weight buffer of qi21_pack_weights: the 15 tensors of qi21_weights in
+// struct order, [out][in] (stacked [L][out][in]), each on a 256-byte boundary.
+struct PackedLayout {
+    size_t off[15];
+    size_t total;
+};
+inline PackedLayout packed_layout(const qi21_config &c) {
+    const size_t eb = dtype_bytes(c.dtype);
+    const size_t d = c.d_model, C = c.latent_ch, T = c.time_dim, F = c.mlp_hidden, L = c.n_layers;
+    const size_t nch = c.use_shift ? 6 : 4, dh = c.head_dim;
+    const size_t sizes[15] = {d * C * eb,     C * d * eb,     d * T * eb,     d * d * eb,     nch * d * d * eb,
+                              d * d * eb,     L * d * d * eb, L * d * d * eb, L * d * d * eb, L * d * d * eb,
+                              L * F * d * eb, L * F * d * eb, L * d * F * eb, L * dh * 4,     L * dh * 4};
+    PackedLayout p{};
+    size_t o = 0;
+    for (int i = 0; i < 15; ++i) {
+        p.off[i] = o;
+        o += align256(sizes[i]);
+    }
+    p.total = o;
+    return p;
+}
+
 inline bool uses_cuda_core_gemm(const qi21_config &c) { return c.dtype == QI21_DTYPE_F32 || !tc_enabled(); }
 
 inline WsLayout ws_layout(const qi21_config &c, int64_t B, int64_t P, int64_t N) {

@@ -210,6 +210,25 @@ __global__ void __launch_bounds__(256) k_img_in64(const float *__restrict__ x, c
 }
 
 // Copy the prefix hidden states [B][P][d] into residual rows b*M_out + n.
+// out[z][c][r] = in[z][r][c] (one matrix per blockIdx.z), 32x32 tiles through
+// shared memory so that both the reads and the writes are coalesced.
+template <typename T>
+__global__ void __launch_bounds__(256) k_transpose(const T *__restrict__ in, T *__restrict__ out, int rows, int cols) {
+    __shared__ T tile[32][33];
+    const size_t mat = (size_t)rows * cols * blockIdx.z;
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    for (int i = ty; i < 32; i += 8) {
+        const int r = r0 + i, c = c0 + tx;
+        if (r < rows && c < cols) tile[i][tx] = in[mat + (size_t)r * cols + c];
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int c = c0 + i, r = r0 + tx;
+        if (r < rows && c < cols) out[mat + (size_t)c * rows + r] = tile[tx][i];
+    }
+}
+
 static __global__ void k_copy_rows(const float *__restrict__ src, float *__restrict__ dst, int rows_per_item, int d,
                             int M_out, int64_t total) {
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;

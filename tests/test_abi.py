@@ -211,3 +211,24 @@ def test_shared_prefix_cache_layout(B):
     w = B.qi21_weights(*([fake] * 15))
     assert B.qi21_cached_step(cfg, w, cache, fake, fake, fake, fake, fake, fake, ws_bytes, 0) == \
         B.QI21_ERR_CACHE_STATE
+
+
+def test_packed_weights_size_and_validation(B):
+    for name in ("small", "full"):
+        sh = C.make_workload(name).shape
+        for dt, eb in ((B.QI21_DTYPE_F32, 4), (B.QI21_DTYPE_BF16, 2)):
+            from prefix_kv_cached_b200.runner import make_config
+            cfg = make_config(sh, dt)
+            want = 0
+            for wname, shp in C.weight_specs(sh):
+                nbytes = int(np.prod(shp)) * (4 if wname in ("q_norm", "k_norm") else eb)
+                want += (nbytes + 255) // 256 * 256
+            assert B.qi21_packed_weights_bytes(cfg) == want
+    cfg = _cfg(B)
+    fake = 0x10000
+    cw = B.qi21_weights_canonical(*([fake] * 15))
+    need = B.qi21_packed_weights_bytes(cfg)
+    assert B.qi21_pack_weights(cfg, cw, fake, need - 1)[0] == B.QI21_ERR_WORKSPACE_TOO_SMALL
+    assert B.qi21_pack_weights(cfg, cw, fake + 8, need)[0] == B.QI21_ERR_INVALID_ARG
+    cw.w_down = fake + 4
+    assert B.qi21_pack_weights(cfg, cw, fake, need)[0] == B.QI21_ERR_INVALID_ARG

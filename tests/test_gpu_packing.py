@@ -89,3 +89,47 @@ def test_packed_prefix_feeds_the_extract(B, mode):
         ck, cv = O.prefix_extract(model, seq, pre_o, m0)
         assert max_rel(gk[:, b], ck) < 1e-4
         assert max_rel(gv[:, b], cv) < 1e-4
+
+
+@pytest.mark.parametrize("dtype_name", ["float32", "bfloat16"])
+def test_pack_weights_from_canonical_layout(B, dtype_name):
+    """qi21_pack_weights: canonical [in][out] weights become exactly the [out][in]
+    tensors the kernels read, and a cached step through them is bit-identical."""
+    from prefix_kv_cached_b200.runner import Qi21Runner
+    w = C.make_workload("small")
+    dtype = B.QI21_DTYPE_F32 if dtype_name == "float32" else B.QI21_DTYPE_BF16
+    _, wts = oracle_model(w, dtype_name)
+    r = Qi21Runner(w, dtype, host_weights=wts)
+    canon = {}
+    for name, _ in C.weight_specs(w.shape):
+        t = r.weights[name]
+        canon[name] = t if name in ("q_norm", "k_norm") else t.transpose(-1, -2).contiguous()
+    cw = B.qi21_weights_canonical(*[canon[n].data_ptr() for n in (
+        "w_img_in", "w_out", "w_t1", "w_t2", "w_mod", "w_fin", "w_q", "w_k", "w_v", "w_o", "w_gate", "w_up",
+        "w_down", "q_norm", "k_norm")])
+    nbytes = B.qi21_packed_weights_bytes(r.cfg)
+    packed = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    st, pw = B.qi21_pack_weights(r.cfg, cw, packed, nbytes)
+    assert st == 0
+    torch.cuda.synchronize()
+    base = packed.data_ptr()
+    for name, shp in C.weight_specs(w.shape):
+        ref = r.weights[name]
+        off = getattr(pw, name) - base
+        got = packed[off: off + ref.numel() * ref.element_size()].view(ref.dtype).view(ref.shape)
+        assert torch.equal(got, ref), name
+    # a cached step through the packed weights equals the step through the original tensors
+    pre = torch.from_numpy(C.host_prefix_hidden(w).astype(np.float32)).cuda()
+    x = torch.from_numpy(C.host_noise(w).astype(np.float32)).cuda()
+    outs = []
+    for wstruct in (r.wstruct, pw):
+        r.wstruct = wstruct
+        v = torch.empty_like(x)
+        r.set_prefix_row()
+        r.prefix_extract(pre)
+        r.set_target_row(w.sigmas[0])
+        r.cached_step(x, v)
+        torch.cuda.synchronize()
+        outs.append(v.clone())
+    r.check_device()
+    assert torch.equal(outs[0], outs[1])
