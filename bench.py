@@ -88,6 +88,10 @@ def kernel_bytes(w):
         "img_in": R * C * 4 + R * d * 4,     # read x, write fp32 h
         "final": R * d * 4 + R * C * 4,      # read h, write v
         "euler": R * C * 12,
+        # modulation: the two GEMV launches of a step read w_t2 (d x d) and then w_mod + w_fin
+        # ((chunks + 1) d x d), bf16; bytes per launch = their mean
+        "gemv": (d * d + (sh.n_chunks + 1) * d * d) * 2 // 2,
+        "temb_in": d * sh.time_dim * 2,
     }
 
 
