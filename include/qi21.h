@@ -254,6 +254,9 @@ qi21_status qi21_modulation_noalloc(const qi21_config *cfg, const qi21_weights *
  *   prefix_hidden  [B][P][d] float32 device (joint hidden states of the prefix)
  *   cos_sin_prefix [P][head_dim/2][2] float32 device
  *   mod_row_prefix [chunks*d] float32 device
+ * With a shared-prefix cache (qi21_kv_cache_init_shared) there is one prefix
+ * for all requests: prefix_hidden is [1][P][d] and rows [0, P) of the single
+ * prefix block are written.
  * On success cache->state = QI21_CACHE_EXTRACTED. */
 qi21_status qi21_prefix_extract(const qi21_config *cfg, const qi21_weights *w,
                                 qi21_kv_cache *cache, const float *prefix_hidden,
@@ -272,7 +275,9 @@ qi21_status qi21_prefix_extract(const qi21_config *cfg, const qi21_weights *w,
  *   mod_row_target [chunks*d], scale_final [d] float32 device (from qi21_modulation)
  *   v_out          [B][N][C] float32 device
  * Returns QI21_ERR_CACHE_STATE unless the cache was extracted with matching
- * sizes. Writes cache rows [P, P+N) (target K/V of this step). */
+ * sizes. Writes cache rows [P, P+N) (target K/V of this step); with a
+ * shared-prefix cache, request b's rows [Pp + b*N, Pp + (b+1)*N), and every
+ * request's attention reads the one copy of the prefix rows. */
 qi21_status qi21_cached_step(const qi21_config *cfg, const qi21_weights *w,
                              const qi21_kv_cache *cache, const float *x_k,
                              const float *cos_sin_target, const float *mod_row_target,
