@@ -39,7 +39,7 @@ UNIT = "target tokens/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--workload", default="full")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -455,7 +455,7 @@ def main():
             bstep(k)
         torch.cuda.synchronize()
         rb.check_device()
-        nb = max(4, args.steps // 2)
+        nb = max(4, min(16, args.steps // 2))
         c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         dist_barrier(world)
         torch.cuda.synchronize()
