@@ -196,11 +196,10 @@ CPU_BASELINE_ROWS = 4096
 REFERENCE_ROWS = 512
 
 
-def oracle_sample(w, rows=REFERENCE_ROWS, seed=4321):
-    """Time the fp64 oracle on a bounded sample of the workload: one block of
-    the cached step at full width for `rows` target tokens attending to all
-    P + N keys (the other targets' K/V are synthetic cache rows). Returns
-    (seconds, target tokens/s scaled to all L blocks, threads, description)."""
+def oracle_sample_inputs(w, rows=REFERENCE_ROWS, seed=4321):
+    """Inputs of the oracle timing sample: one block of the cached step at full
+    width for `rows` target tokens attending to all P + N keys (the other
+    targets' K/V are synthetic cache rows). Drawn once, reused by every timed run."""
     from oracle import qi21_oracle as O
 
     rows = min(rows, w.n_target)
@@ -208,31 +207,38 @@ def oracle_sample(w, rows=REFERENCE_ROWS, seed=4321):
     d, F, H, Dh = sh.d_model, sh.mlp_hidden, sh.n_heads, sh.head_dim
     rng = np.random.default_rng(seed)   # timing sample only: values are not compared with anything
 
-    def draw(name, shape, std):
+    def draw(shape, std):
         return rng.standard_normal(shape) * std
 
-    lw = {"w_q": draw("wq", (d, d), 0.02), "w_k": draw("wk", (d, d), 0.02), "w_v": draw("wv", (d, d), 0.02),
-          "w_o": draw("wo", (d, d), 0.02), "w_gate": draw("wg", (F, d), 0.02), "w_up": draw("wu", (F, d), 0.02),
-          "w_down": draw("wd", (d, F), 0.02), "q_norm": draw("qn", (Dh,), 0.02), "k_norm": draw("kn", (Dh,), 0.02)}
+    lw = {"w_q": draw((d, d), 0.02), "w_k": draw((d, d), 0.02), "w_v": draw((d, d), 0.02),
+          "w_o": draw((d, d), 0.02), "w_gate": draw((F, d), 0.02), "w_up": draw((F, d), 0.02),
+          "w_down": draw((d, F), 0.02), "q_norm": draw((Dh,), 0.02), "k_norm": draw((Dh,), 0.02)}
     extra = w.n_prefix + w.n_target - rows
-    kc = draw("kc", (extra, H, Dh), 1.0)
-    vc = draw("vc", (extra, H, Dh), 1.0)
-    h = draw("h", (rows, d), 1.0)
-    mods = O.split_chunks(draw("mod", (4 * d,), 0.1), 4)
-    coords = O.rope_coords(w.segments)[w.n_prefix:w.n_prefix + rows]
-    omega = O.rope_omega_axial(Dh)
-    allowed = np.ones((rows, extra + rows), dtype=bool)
+    return {"rows": rows, "lw": lw, "kc": draw((extra, H, Dh), 1.0), "vc": draw((extra, H, Dh), 1.0),
+            "h": draw((rows, d), 1.0), "mods": O.split_chunks(draw((4 * d,), 0.1), 4),
+            "coords": O.rope_coords(w.segments)[w.n_prefix:w.n_prefix + rows],
+            "omega": O.rope_omega_axial(Dh), "allowed": np.ones((rows, extra + rows), dtype=bool)}
+
+
+def oracle_sample(w, rows=REFERENCE_ROWS, seed=4321, inputs=None):
+    """Time the fp64 oracle on the bounded sample of oracle_sample_inputs. Returns
+    (seconds, target tokens/s scaled to all L blocks, threads, description)."""
+    from oracle import qi21_oracle as O
+
+    sh = w.shape
+    x = inputs if inputs is not None else oracle_sample_inputs(w, rows, seed)
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    O.dit_block(h, mods, lw, H, coords, omega, (kc, vc), allowed, sh.ln_eps, sh.qk_eps)
+    O.dit_block(x["h"], x["mods"], x["lw"], sh.n_heads, x["coords"], x["omega"], (x["kc"], x["vc"]), x["allowed"],
+                sh.ln_eps, sh.qk_eps)
     dt = time.perf_counter() - t0
-    tok_s = rows / (dt * sh.n_layers)
-    desc = (f"one of {sh.n_layers} blocks of the cached step at d={d}, {rows} target rows attending to "
-            f"{w.n_prefix + w.n_target} keys, fp64 numpy; time x {sh.n_layers} blocks per token")
+    tok_s = x["rows"] / (dt * sh.n_layers)
+    desc = (f"one of {sh.n_layers} blocks of the cached step at d={sh.d_model}, {x['rows']} target rows attending "
+            f"to {w.n_prefix + w.n_target} keys, fp64 numpy; time x {sh.n_layers} blocks per token")
     return dt, tok_s, threads, desc
 
 
@@ -288,8 +294,9 @@ def run_reference(args, w, world, rank):
         return 0
     steps = []
     desc = threads = None
+    inputs = oracle_sample_inputs(w)
     for i in range(args.warmup + args.steps):
-        dt, tok_s, threads, desc = oracle_sample(w)
+        dt, tok_s, threads, desc = oracle_sample(w, inputs=inputs)
         if i >= args.warmup:
             steps.append(dt)
     dt = statistics.mean(steps)
