@@ -47,7 +47,11 @@ reason in the design notes of the repository):
   PACK_ADD).
 
 Parity unpinned: nothing. Each function has a pin in ``tests/test_oracle_pins.py``
-(page-printed values, closed forms, library routines or brute force).
+(page-printed values, closed forms, library routines or brute force); the
+output head (``final_velocity``, ``img_in``), which the lab replay's drift
+check never reaches, is pinned by closed-form LayerNorm rows through a
+non-symmetric one-hot W_out and by hand-worked products, and
+``tests/test_oracle_mutations.py`` shows each pin catching planted mistakes.
 """
 from __future__ import annotations
 
@@ -513,20 +517,22 @@ def cached_step(model: Model, seq: Sequence_, cache_k: np.ndarray, cache_v: np.n
 
     Only the target rows run the blocks; their keys are [cached prefix; own].
     The target rows' mask row allows all P + N keys (target is last).
-    Returns (v [N, C], target K [L, N, H, Dh]).
+    Returns (v [N, C], target K [L, N, H, Dh], target V [L, N, H, Dh]): the K/V
+    rows this step appends to each layer's cache after the prefix.
     """
     p, n = seq.P, seq.N
     mods = split_chunks(mod_target, model.n_chunks)
     h = img_in(x, model.wts["w_img_in"])
     allowed = seq.allowed[p:, :]
-    tk = []
+    tk, tv = [], []
     for l in range(model.n_layers):
         out = dit_block(h, mods, layer_weights(model.wts, l), model.n_heads, seq.coords[p:],
                         model.omega, (cache_k[l], cache_v[l]), allowed, model.ln_eps, model.qk_eps)
         h = out.h
         tk.append(out.k_rot)
+        tv.append(out.v)
     v = final_velocity(h, scale_final, model.wts["w_out"], model.ln_eps)
-    return v, np.stack(tk)
+    return v, np.stack(tk), np.stack(tv)
 
 
 def run_image(model: Model, seq: Sequence_, prefix_hidden: np.ndarray, x0: np.ndarray,
@@ -554,7 +560,7 @@ def run_image(model: Model, seq: Sequence_, prefix_hidden: np.ndarray, x0: np.nd
         if use_cache and k == 0:
             ck, cv = prefix_extract(model, seq, prefix_hidden, mod_p)
         if use_cache:
-            v, _ = cached_step(model, seq, ck, cv, x, mod_t, sf)
+            v = cached_step(model, seq, ck, cv, x, mod_t, sf)[0]
             modes.append("extract" if k == 0 else "cached")
         else:
             v = joint_forward(model, seq, prefix_hidden, x, mod_p, mod_t, sf)["v"]

@@ -112,3 +112,26 @@ def test_packing_pins_catch_mutation(monkeypatch, fname, old, new):
         except (AssertionError, IndexError, ValueError):   # a pin that fails or breaks catches it
             failed += 1
     assert failed > 0, f"mutation in {fname} not caught by any packing pin"
+
+
+HEAD_MUTATIONS = [
+    ("final_velocity", "(1.0 + scale_final)", "(scale_final)"),                          # dropped 1 +
+    ("final_velocity", "(1.0 + scale_final))", "(1.0 + scale_final) + scale_final)"),    # added shift
+    ("final_velocity", "@ w_out.T", "@ w_out"),                                          # transposed W_out
+    ("final_velocity", "layernorm(h_target, ln_eps)", "h_target"),                       # LN dropped
+    ("img_in", "return x @ w_img_in.T", "return 2.0 * (x @ w_img_in.T)"),                # doubled img_in
+    ("img_in", "return x @ w_img_in.T", "return x @ w_img_in[::-1].T"),                  # wrong row order
+]
+
+
+@pytest.mark.parametrize("fname,old,new", HEAD_MUTATIONS, ids=[f"{m[0]}:{i}" for i, m in enumerate(HEAD_MUTATIONS)])
+def test_head_pins_catch_mutation(monkeypatch, fname, old, new):
+    from tests import test_oracle_pins as P
+    monkeypatch.setattr(O, fname, _mutant(getattr(O, fname), old, new))
+    failed = 0
+    for pin in (P.test_final_velocity_closed_forms, P.test_img_in_hand_worked):
+        try:
+            pin()
+        except (AssertionError, ValueError):
+            failed += 1
+    assert failed > 0, f"mutation in {fname} not caught by the output-head pins"

@@ -227,6 +227,43 @@ def test_attention_special_cases():
     np.testing.assert_allclose(same[0], np.repeat(v[0].mean(axis=0, keepdims=True), 3, 0), atol=1e-15)
 
 
+# ---------------------------------------------------------------- output head and img_in
+
+def test_final_velocity_closed_forms():
+    """6B page §1 and §3: v = (LN(h)(1 + scale_final)) W_out, scale-only (no
+    shift, no bias). Two rows whose LayerNorm is known in closed form:
+    an alternating row (+a, -a, ...) has mean 0 and variance a^2, so LN gives
+    +-a / sqrt(a^2 + eps); the row 1, 2, ..., 8 has mean 4.5 and biased
+    variance (8^2 - 1) / 12 = 5.25. W_out picks dimension (c + 1) mod 8 for
+    output c (a cyclic shift, so W_out and its transpose differ), which makes
+    v[c] = LN(h)[j] (1 + s[j]) with j = (c + 1) mod 8."""
+    d, a, eps = 8, 2.0, 1e-6
+    h = np.array([[a, -a] * 4, list(range(1, 9))], dtype=np.float64)
+    s = np.array([0.5, -0.25, 2.0, 0.0, -1.5, 0.75, 1.0, -0.5])
+    w_out = np.zeros((d, d))
+    for c in range(d):
+        w_out[c, (c + 1) % d] = 1.0
+    ln0 = np.array([1.0, -1.0] * 4) * a / math.sqrt(a * a + eps)
+    ln1 = (np.arange(1, 9) - 4.5) / math.sqrt(5.25 + eps)
+    for row, ln in ((0, ln0), (1, ln1)):
+        want = np.array([ln[(c + 1) % d] * (1.0 + s[(c + 1) % d]) for c in range(d)])
+        np.testing.assert_allclose(O.final_velocity(h[row:row + 1], s, w_out, eps)[0], want, rtol=1e-13,
+                                   atol=1e-15)
+    # scale_final = 0 leaves the plain LayerNorm through W_out
+    np.testing.assert_allclose(O.final_velocity(h[1:], np.zeros(d), w_out, eps)[0], np.roll(ln1, -1),
+                               rtol=1e-13)
+
+
+def test_img_in_hand_worked():
+    """img_in with patch size 1 (lab [1A]; End-to-end lab §3): token = latent
+    times W_img_in^T, W_img_in [d][C]. Worked by hand for C = 3, d = 4."""
+    x = np.array([[1.0, 2.0, 3.0], [0.0, -1.0, 2.0]])
+    w_img_in = np.array([[1.0, 0.0, 0.0], [0.0, 1.0, 0.0], [0.0, 0.0, 1.0], [1.0, 1.0, 1.0]])
+    np.testing.assert_array_equal(O.img_in(x, w_img_in), np.array([[1.0, 2.0, 3.0, 6.0], [0.0, -1.0, 2.0, 1.0]]))
+    w2 = np.array([[2.0, -1.0, 0.5], [0.0, 0.0, 0.0], [1.0, 1.0, -1.0], [0.0, 3.0, 0.0]])
+    np.testing.assert_array_equal(O.img_in(x, w2), np.array([[1.5, 0.0, 0.0, 6.0], [2.0, 0.0, -3.0, -3.0]]))
+
+
 # ---------------------------------------------------------------- modulation
 
 def test_timestep_embedding_closed_forms():
