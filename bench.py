@@ -346,7 +346,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     seed_w = C.Workload(w.name, w.shape, w.batch, w.segments, w.sigmas, w.seed + 1000 * rank)
-    r = Qi21Runner(seed_w, B.QI21_DTYPE_BF16, device=str(dev))
+    r = Qi21Runner(seed_w, B.QI21_DTYPE_BF16, device=str(dev),
+                   weights=C.device_weights(seed_w, torch.bfloat16, dev))
     sh = w.shape
     pre = normal_torch(seed_w.seed, "prefix_hidden", (w.batch, w.n_prefix, sh.d_model), device=dev,
                        dtype=torch.float32)

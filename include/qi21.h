@@ -191,7 +191,15 @@ qi21_status qi21_build_packing(const qi21_segment *segments, int32_t n_segments,
                                int32_t *slot_of, int32_t *img_row, int32_t *P,
                                int32_t *n_slots, int32_t *n_img);
 
-/* Sin-cos timestep embedding [time_dim]/* Sin-cos timestep embedding [time_dim] (host, fp64 math, float result):
+/* The lab's micro RoPE split for head_dim 4 ([LAB] 3A), omega [2][3] (host):
+ * pair 0 turns with the frame axis at rate 1; pair 1 is shared by height
+ * (rate base^-1) and width (rate base^-1.5), the two angles adding. */
+qi21_status qi21_rope_omega_lab(double base, double *omega);
+
+/* Timestep of a noise level: t = QI21_T_PER_SIGMA * sigma ([3B] §1; [6B] §3). */
+#define QI21_T_PER_SIGMA 1000.0
+
+/* Sin-cos timestep embedding [time_dim] (host, fp64 math, float result):
  * [cos(t f_i) ..., sin(t f_i) ...], f_i = 10000^(-2i/time_dim), t = 1000*sigma
  * ([LAB] 3B, [3B] §1). */
 qi21_status qi21_timestep_embedding(double t, int32_t time_dim, float *emb);
@@ -224,6 +232,12 @@ qi21_status qi21_kv_cache_init_shared(qi21_kv_cache *cache, void *base, const qi
 qi21_status qi21_modulation(const qi21_config *cfg, const qi21_weights *w, double t,
                             float *mod_row, float *scale_final,
                             void *ws, size_t ws_bytes, void *stream);
+
+/* qi21_modulation at the timestep of noise level sigma, t = QI21_T_PER_SIGMA * sigma
+ * (formed on the host in fp64). */
+qi21_status qi21_modulation_sigma(const qi21_config *cfg, const qi21_weights *w, double sigma,
+                                  float *mod_row, float *scale_final,
+                                  void *ws, size_t ws_bytes, void *stream);
 
 /* Largest d_model qi21_modulation_noalloc accepts: its scratch is a fixed
  * device array of 2 * QI21_NOALLOC_MAX_D floats (64 KB on every GPU that
@@ -339,7 +353,7 @@ qi21_status qi21_pack_prefix(int32_t batch, int32_t P, int32_t d, int32_t n_slot
 qi21_status qi21_img_in_tokens(const qi21_config *cfg, const qi21_weights *w, const float *latents,
                                int32_t rows, float *out, void *stream);
 
-/* Device-indexed forms for captured sequences (CUDA graphs)/* Device-indexed forms for captured sequences (CUDA graphs): the sigma of a
+/* Device-indexed forms for captured sequences (CUDA graphs): the sigma of a
  * step is read on the device from sigmas, a table of float64 values in device
  * memory (8-byte aligned, caller-owned, at least step + 2 entries), so one
  * captured sequence serves any sigma schedule written into the table before a
@@ -411,6 +425,17 @@ void qi21_profile_reset(void);
  * and attention; 0 the CUDA-core kernels of the F32 mode run on bf16 storage
  * (differential testing of the two families). Process-wide. */
 void qi21_set_tensor_cores(int32_t enable);
+
+/* Kernel family the block stack of cfg runs on under the current setting:
+ * QI21_FAMILY_TENSOR_CORES (BF16 with tensor cores enabled and a supported
+ * shape), QI21_FAMILY_CUDA_CORES (F32, or BF16 with tensor cores switched
+ * off), or QI21_FAMILY_NONE when the entry points refuse cfg (an invalid
+ * config, or a BF16 shape the tensor-core kernels do not cover: d_model a
+ * multiple of 256, head_dim 64 or 128, mlp_hidden a multiple of 128). BF16
+ * never falls back to the CUDA-core kernels on its own: such a config returns
+ * QI21_ERR_UNSUPPORTED from every device entry point. */
+enum { QI21_FAMILY_NONE = -1, QI21_FAMILY_CUDA_CORES = 0, QI21_FAMILY_TENSOR_CORES = 1 };
+int32_t qi21_kernel_family(const qi21_config *cfg);
 
 /* Library version string and the number of kernels the last entry point call
  * enqueued (for launch accounting). */

@@ -31,6 +31,10 @@ QI21_SEG_TEXT = 0
 QI21_SEG_IMAGE = 1
 QI21_CACHE_EMPTY = 0
 QI21_CACHE_EXTRACTED = 1
+QI21_FAMILY_NONE = -1
+QI21_FAMILY_CUDA_CORES = 0
+QI21_FAMILY_TENSOR_CORES = 1
+QI21_T_PER_SIGMA = 1000.0
 
 
 class qi21_config(ct.Structure):
@@ -71,6 +75,7 @@ _SIGS = {
     "qi21_build_metadata": (_I32, [ct.POINTER(qi21_segment), _I32, _I32, _I32, _P, _P, _P, _P,
                                    ct.POINTER(_I32), ct.POINTER(_I32), ct.POINTER(_I32)]),
     "qi21_rope_omega_axial": (_I32, [_I32, ct.c_double, _P]),
+    "qi21_rope_omega_lab": (_I32, [ct.c_double, _P]),
     "qi21_rope_table": (_I32, [_I32, _P, _I32, _P, _P]),
     "qi21_timestep_embedding": (_I32, [ct.c_double, _I32, _P]),
     "qi21_kv_cache_bytes": (ct.c_size_t, [ct.POINTER(qi21_config), _I32, _I32, _I32]),
@@ -84,6 +89,8 @@ _SIGS = {
                                          _I32]),
     "qi21_modulation": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P, _P,
                                ct.c_size_t, _P]),
+    "qi21_modulation_sigma": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P, _P,
+                                     ct.c_size_t, _P]),
     "qi21_modulation_noalloc": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.c_double, _P, _P,
                                        _P]),
     "qi21_prefix_extract": (_I32, [ct.POINTER(qi21_config), ct.POINTER(qi21_weights), ct.POINTER(qi21_kv_cache),
@@ -111,6 +118,7 @@ _SIGS = {
     "qi21_version": (ct.c_char_p, []),
     "qi21_last_launch_count": (_I32, []),
     "qi21_set_tensor_cores": (None, [_I32]),
+    "qi21_kernel_family": (_I32, [ct.POINTER(qi21_config)]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -178,6 +186,13 @@ def qi21_rope_omega_axial(head_dim, base=10000.0):
     return om
 
 
+def qi21_rope_omega_lab(base=10000.0):
+    import numpy as np
+    om = np.zeros((2, 3), np.float64)
+    check("qi21_rope_omega_lab", lib.qi21_rope_omega_lab(base, _addr(om)))
+    return om
+
+
 def qi21_rope_table(head_dim, coords, omega):
     import numpy as np
     coords = np.ascontiguousarray(coords, dtype=np.int32)
@@ -234,6 +249,11 @@ def qi21_kv_cache_init_shared(base, cfg, batch, n_prefix, n_target):
 def qi21_modulation(cfg, weights, t, mod_row, scale_final, ws, ws_bytes, stream=0):
     return lib.qi21_modulation(ct.byref(cfg), ct.byref(weights), float(t), _addr(mod_row), _addr(scale_final),
                                _addr(ws), ws_bytes, stream)
+
+
+def qi21_modulation_sigma(cfg, weights, sigma, mod_row, scale_final, ws, ws_bytes, stream=0):
+    return lib.qi21_modulation_sigma(ct.byref(cfg), ct.byref(weights), float(sigma), _addr(mod_row),
+                                     _addr(scale_final), _addr(ws), ws_bytes, stream)
 
 
 def qi21_modulation_noalloc(cfg, weights, t, mod_row, scale_final, stream=0):
@@ -354,3 +374,7 @@ def qi21_last_launch_count():
 
 def qi21_set_tensor_cores(on):
     lib.qi21_set_tensor_cores(1 if on else 0)
+
+
+def qi21_kernel_family(cfg):
+    return int(lib.qi21_kernel_family(ct.byref(cfg)))

@@ -581,6 +581,18 @@ extern "C" qi21_status qi21_modulation(const qi21_config *c, const qi21_weights 
     return modulation_impl(c, w, &emb, nullptr, 0, 0.0, mod_row, scale_final, ws, ws_bytes, stream);
 }
 
+extern "C" qi21_status qi21_modulation_sigma(const qi21_config *c, const qi21_weights *w, double sigma,
+                                             float *mod_row, float *scale_final, void *ws, size_t ws_bytes,
+                                             void *stream) {
+    if (!std::isfinite(sigma)) return QI21_ERR_INVALID_ARG;
+    return qi21_modulation(c, w, QI21_T_PER_SIGMA * sigma, mod_row, scale_final, ws, ws_bytes, stream);
+}
+
+extern "C" int32_t qi21_kernel_family(const qi21_config *c) {
+    if (check_shapes(c) != QI21_OK) return QI21_FAMILY_NONE;
+    return uses_cuda_core_gemm(*c) ? QI21_FAMILY_CUDA_CORES : QI21_FAMILY_TENSOR_CORES;
+}
+
 extern "C" qi21_status qi21_modulation_at(const qi21_config *c, const qi21_weights *w, const double *sigmas,
                                           int32_t step, double t_per_sigma, float *mod_row, float *scale_final,
                                           void *ws, size_t ws_bytes, void *stream) {

@@ -81,6 +81,15 @@ extern "C" qi21_status qi21_rope_omega_axial(int32_t head_dim, double base, doub
     return p == head_dim / 2 ? QI21_OK : QI21_ERR_SHAPE;
 }
 
+extern "C" qi21_status qi21_rope_omega_lab(double base, double *omega) {
+    // [LAB] 3A micro split: pair 0 = frame at rate 1; pair 1 = height at
+    // base^-1 plus width at base^-1.5.
+    if (!omega || !(base > 1.0)) return QI21_ERR_INVALID_ARG;
+    const double v[6] = {1.0, 0.0, 0.0, 0.0, std::pow(base, -1.0), std::pow(base, -1.5)};
+    std::memcpy(omega, v, sizeof(v));
+    return QI21_OK;
+}
+
 extern "C" qi21_status qi21_rope_table(int32_t head_dim, const int32_t *coords, int32_t S,
                                        const double *omega, float *cos_sin) {
     if (!coords || !omega || !cos_sin || head_dim <= 0 || head_dim % 2 || S < 0) return QI21_ERR_INVALID_ARG;

@@ -1,43 +1,48 @@
 """Device-side driver of one model instance over the C ABI.
 
-Owns the torch-allocated device buffers (weights, K/V cache, workspace,
-metadata tables) and calls the library's entry points; it computes nothing
-itself. Weights come either from host arrays (exact stored values) or are
-drawn directly on the device with the seeded generator (large models).
+Owns the torch-allocated device buffers (K/V cache, workspace, metadata
+tables, modulation rows) and calls the library's entry points; it computes
+nothing itself. The caller supplies the weights, either as host arrays (copied
+to the device once) or as device tensors it already holds, and a description
+of the model and the sequence: an object with ``shape`` (the fields of
+``qi21_config`` plus ``rope``: "axial" or "lab"), ``segments`` (kind, n_text | h,
+w), ``batch``, ``n_prefix`` and ``n_target``.
 """
 from __future__ import annotations
 
-import math
 from typing import Dict, Optional
 
 import numpy as np
 import torch
 
 from . import binding as B
-from qi21_synth import configs as C
-from qi21_synth.gen import normal_torch
 
 _TORCH_DTYPE = {B.QI21_DTYPE_F32: torch.float32, B.QI21_DTYPE_BF16: torch.bfloat16}
 
+# qi21_weights field order
+WEIGHT_NAMES = ("w_img_in", "w_out", "w_t1", "w_t2", "w_mod", "w_fin", "w_q", "w_k", "w_v", "w_o", "w_gate",
+                "w_up", "w_down", "q_norm", "k_norm")
+NORM_WEIGHTS = ("q_norm", "k_norm")      # float32 in both storage modes
 
-def make_config(shape: C.ModelShape, dtype: int) -> B.qi21_config:
+
+def make_config(shape, dtype: int) -> B.qi21_config:
     return B.qi21_config(shape.d_model, shape.n_heads, shape.head_dim, shape.n_layers, shape.mlp_hidden,
                          shape.latent_ch, shape.time_dim, dtype, shape.use_shift, shape.ln_eps, shape.qk_eps)
 
 
-def lab_rope_omega(base: float = 10000.0) -> np.ndarray:
-    """Micro RoPE split of the lab (head_dim 4): pair 0 on the frame axis at
-    rate 1; pair 1 shared by height (base^-1) and width (base^-1.5)."""
-    return np.array([[1.0, 0.0, 0.0], [0.0, base ** -1.0, base ** -1.5]], dtype=np.float64)
-
-
 class Qi21Runner:
-    def __init__(self, workload: C.Workload, dtype: int = B.QI21_DTYPE_F32, device: str = "cuda",
-                 host_weights: Optional[Dict[str, np.ndarray]] = None, frame_mode: int = 0,
+    def __init__(self, workload, dtype: int = B.QI21_DTYPE_F32, device: str = "cuda",
+                 host_weights: Optional[Dict[str, np.ndarray]] = None,
+                 weights: Optional[Dict[str, torch.Tensor]] = None, frame_mode: int = 0,
                  shared_prefix: bool = False, share_weights_with: Optional["Qi21Runner"] = None):
-        """shared_prefix: the batch items are requests sharing one prefix (one
-        extract from prefix_hidden [1][P][d], every request's attention reading
-        the one copy); share_weights_with: reuse another runner's device weights."""
+        """Weights: exactly one of host_weights (arrays holding the stored values,
+        copied to the device in the storage dtype), weights (device tensors in the
+        storage dtype, norm weights float32) or share_weights_with (another
+        runner's device weights). shared_prefix: the batch items are requests
+        sharing one prefix (one extract from prefix_hidden [1][P][d], every
+        request's attention reading the one copy)."""
+        if sum(x is not None for x in (host_weights, weights, share_weights_with)) != 1:
+            raise ValueError("give exactly one of host_weights, weights, share_weights_with")
         self.w = workload
         self.shape = workload.shape
         self.dtype = dtype
@@ -49,7 +54,7 @@ class Qi21Runner:
         self.S, self.P, self.N = self.meta["S"], self.meta["P"], self.meta["N"]
         assert (self.P, self.N) == (workload.n_prefix, workload.n_target)
         self.Bn = workload.batch
-        omega = lab_rope_omega() if sh.rope == "lab" else B.qi21_rope_omega_axial(sh.head_dim)
+        omega = B.qi21_rope_omega_lab() if sh.rope == "lab" else B.qi21_rope_omega_axial(sh.head_dim)
         cs = B.qi21_rope_table(sh.head_dim, self.meta["coords"], omega)
         self.cos_sin_all = torch.from_numpy(cs).to(self.device)
         self.cos_sin_prefix = self.cos_sin_all[: self.P].contiguous()
@@ -59,19 +64,18 @@ class Qi21Runner:
         self.kv_limit_prefix = lim[: self.P].contiguous()
         self.weights: Dict[str, torch.Tensor] = {}
         self.shared_prefix = shared_prefix
-        for name, shp in C.weight_specs(sh):
+        for name in WEIGHT_NAMES:
+            sdt = torch.float32 if name in NORM_WEIGHTS else self.tdtype
             if share_weights_with is not None:
-                self.weights[name] = share_weights_with.weights[name]
-                continue
-            sdt = torch.float32 if name in ("q_norm", "k_norm") else self.tdtype
-            if host_weights is not None:
-                self.weights[name] = torch.from_numpy(np.ascontiguousarray(host_weights[name])).to(
-                    device=self.device, dtype=sdt)
+                t = share_weights_with.weights[name]
+            elif weights is not None:
+                t = weights[name]
             else:
-                self.weights[name] = self._draw_weight(name, shp, sdt)
-        self.wstruct = B.qi21_weights(*[self.weights[n].data_ptr() for n in (
-            "w_img_in", "w_out", "w_t1", "w_t2", "w_mod", "w_fin", "w_q", "w_k", "w_v", "w_o", "w_gate", "w_up",
-            "w_down", "q_norm", "k_norm")])
+                t = torch.from_numpy(np.ascontiguousarray(host_weights[name])).to(device=self.device, dtype=sdt)
+            if t.dtype != sdt or t.device != self.device or not t.is_contiguous():
+                raise ValueError(f"weight {name}: expected a contiguous {sdt} tensor on {self.device}")
+            self.weights[name] = t
+        self.wstruct = B.qi21_weights(*[self.weights[n].data_ptr() for n in WEIGHT_NAMES])
         if shared_prefix:
             kvb = B.qi21_kv_cache_bytes_shared(self.cfg, self.Bn, self.P, self.N)
             self.cache_buf = torch.zeros(kvb, dtype=torch.uint8, device=self.device)
@@ -82,22 +86,11 @@ class Qi21Runner:
             self.cache = B.qi21_kv_cache_init(self.cache_buf, self.cfg, self.Bn, self.P, self.N)
         self.ws_bytes = B.qi21_workspace_bytes(self.cfg, self.Bn, self.P, self.N)
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.device)
-        nch = sh.n_chunks
+        nch = 6 if sh.use_shift else 4
         self.mod_prefix = torch.zeros(nch * sh.d_model, dtype=torch.float32, device=self.device)
         self.mod_target = torch.zeros_like(self.mod_prefix)
         self.scale_final = torch.zeros(sh.d_model, dtype=torch.float32, device=self.device)
         self._sf0 = torch.zeros_like(self.scale_final)
-
-    def _draw_weight(self, name, shp, sdt):
-        w = self.w
-        if len(shp) == 3 or name in ("q_norm", "k_norm"):
-            out = torch.empty(shp, dtype=sdt, device=self.device)
-            for l in range(shp[0]):
-                out[l] = normal_torch(w.seed, f"L{l}.{name}", shp[1:], std=w.weight_std, device=self.device,
-                                      dtype=torch.float32).to(sdt)
-            return out
-        return normal_torch(w.seed, name, shp, std=w.weight_std, device=self.device,
-                            dtype=torch.float32).to(sdt)
 
     @property
     def stream(self) -> int:
@@ -113,7 +106,11 @@ class Qi21Runner:
         self.modulation(0.0, self.mod_prefix, self._sf0)
 
     def set_target_row(self, sigma: float):
-        self.modulation(1000.0 * float(sigma), self.mod_target, self.scale_final)
+        """Target modulation row and final scale at noise level sigma (the library
+        forms t = QI21_T_PER_SIGMA * sigma)."""
+        B.check("qi21_modulation_sigma", B.qi21_modulation_sigma(self.cfg, self.wstruct, float(sigma),
+                                                                 self.mod_target, self.scale_final, self.ws,
+                                                                 self.ws_bytes, self.stream))
 
     def prefix_extract(self, prefix_hidden: torch.Tensor, mod_prefix: Optional[torch.Tensor] = None):
         B.check("qi21_prefix_extract", B.qi21_prefix_extract(
@@ -136,8 +133,6 @@ class Qi21Runner:
         B.check("qi21_euler_update", B.qi21_euler_update(x, v, s0, s1, x_out, x.numel(), self.stream))
 
     # ------------------------------------------------------------------ whole image
-    # t = 1000 * sigma (3B page §1; 6B page §3)
-    T_PER_SIGMA = 1000.0
 
     def denoise_image(self, prefix_hidden: torch.Tensor, x: torch.Tensor, sigmas_dev: torch.Tensor,
                       v: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -148,7 +143,7 @@ class Qi21Runner:
         v = torch.empty_like(x) if v is None else v
         B.check("qi21_denoise_image", B.qi21_denoise_image(
             self.cfg, self.wstruct, self.cache, prefix_hidden, self.cos_sin_prefix, self.kv_limit_prefix,
-            self.cos_sin_target, sigmas_dev, sigmas_dev.numel() - 1, self.T_PER_SIGMA, x, v, self.mod_prefix,
+            self.cos_sin_target, sigmas_dev, sigmas_dev.numel() - 1, B.QI21_T_PER_SIGMA, x, v, self.mod_prefix,
             self.mod_target, self.scale_final, self.ws, self.ws_bytes, self.stream))
         return x
 

@@ -232,3 +232,26 @@ def test_packed_weights_size_and_validation(B):
     assert B.qi21_pack_weights(cfg, cw, fake + 8, need)[0] == B.QI21_ERR_INVALID_ARG
     cw.w_down = fake + 4
     assert B.qi21_pack_weights(cfg, cw, fake, need)[0] == B.QI21_ERR_INVALID_ARG
+
+
+def test_bf16_shape_without_tensor_core_kernels_is_refused(B):
+    """BF16 never falls back to the CUDA-core kernels on its own: a head_dim the
+    tensor-core attention does not cover is refused before any launch."""
+    from prefix_kv_cached_b200.runner import make_config
+    shape = C.ModelShape(256, 8, 32, 1, 768, 64, 256)
+    cfg = make_config(shape, B.QI21_DTYPE_BF16)
+    assert B.qi21_kernel_family(cfg) == B.QI21_FAMILY_NONE
+    fake = 0x10000
+    w = B.qi21_weights(*([fake] * 15))
+    cache = B.qi21_kv_cache(fake, 1, 8, 8, 1, 256, B.QI21_DTYPE_BF16, B.QI21_CACHE_EXTRACTED, 0)
+    st = B.qi21_cached_step(cfg, w, cache, fake, fake, fake, fake, fake, fake, 1 << 30, 0)
+    assert st == B.QI21_ERR_UNSUPPORTED
+    B.qi21_set_tensor_cores(0)
+    try:
+        assert B.qi21_kernel_family(cfg) == B.QI21_FAMILY_CUDA_CORES
+    finally:
+        B.qi21_set_tensor_cores(1)
+
+
+def test_lab_rope_omega_matches_oracle(B):
+    assert np.array_equal(B.qi21_rope_omega_lab(), O.rope_omega_lab())

@@ -11,12 +11,10 @@ import torch
 
 from oracle import qi21_oracle as O
 from qi21_synth import configs as C
-from tests._harness import oracle_model, max_rel, rel_l2
+from tests._harness import (BF16_TOL, F32_TOL, assert_item_matches, gpu_steps, max_rel, oracle_item,
+                            oracle_model, rel_l2)
 
 pytestmark = pytest.mark.gpu
-
-F32_TOL = 1e-4
-BF16_TOL = 2e-2
 
 
 @pytest.fixture(scope="module")
@@ -39,7 +37,7 @@ def _oracle_image(model, seq, pre, x0, sigmas, n_steps):
     vs, xs = [], []
     for k in range(n_steps):
         mt, sf = O.modulation(1000.0 * sigmas[k], model.wts, model.n_chunks)
-        v, _ = O.cached_step(model, seq, ck, cv, x, mt, sf)
+        v = O.cached_step(model, seq, ck, cv, x, mt, sf)[0]
         x = O.euler_step(x, v, sigmas[k], sigmas[k + 1])
         vs.append(v)
         xs.append(x)
@@ -63,29 +61,24 @@ def _gpu_image(r, pre_t, x0_t, sigmas, n_steps):
     return vs, xs
 
 
-@pytest.mark.parametrize("name,n_steps", [("toy", 3), ("small", 8), ("small64", 3)])
+@pytest.mark.parametrize("name,n_steps", [("toy", 3), ("toy_parity", 3), ("small", 8), ("small64", 3)])
 def test_f32_denoise_matches_oracle(B, name, n_steps):
-    w = C.make_workload(name)
+    """Every layer's prefix K/V, every step's target K/V of every layer, v_theta
+    and the latent, F32 storage within 1e-4 max relative error. toy is the
+    lab-scale configuration with N(0, 0.02) weights; toy_parity the same shape
+    with the parity weight recipe."""
+    w = C.parity_workload("toy") if name == "toy_parity" else C.make_workload(name)
     model, wts = oracle_model(w, "float32")
     seq = O.make_sequence(w.segments)
     pre = C.host_prefix_hidden(w)
     x0 = C.host_noise(w)
     r = _runner(w, B.QI21_DTYPE_F32, wts)
-    pre_t = torch.from_numpy(pre.astype(np.float32)).cuda()
-    x0_t = torch.from_numpy(x0.astype(np.float32)).cuda()
-    gvs, gxs = _gpu_image(r, pre_t, x0_t, w.sigmas, n_steps)
-    K, V = r.cache_kv()
+    got = gpu_steps(r, torch.from_numpy(pre.astype(np.float32)).cuda(),
+                    torch.from_numpy(x0.astype(np.float32)).cuda(), w.sigmas, n_steps)
     for b in range(w.batch):
-        ck, cv, vs, xs, m0 = _oracle_image(model, seq, pre[b], x0[b], w.sigmas, n_steps)
-        # prefix cache rows, every layer
-        gk = K[:, b, :seq.P].double().cpu().numpy()
-        gv = V[:, b, :seq.P].double().cpu().numpy()
-        assert max_rel(gk, ck) < F32_TOL
-        assert max_rel(gv, cv) < F32_TOL
-        for k in range(n_steps):
-            assert max_rel(gvs[k][b], vs[k]) < F32_TOL, f"v step {k} item {b}"
-            assert max_rel(gxs[k][b], xs[k]) < F32_TOL, f"x step {k} item {b}"
-    assert max_rel(r.mod_prefix.double().cpu().numpy(), m0) < F32_TOL
+        want = oracle_item(model, seq, pre[b], x0[b], w.sigmas, n_steps)
+        assert_item_matches(got, want, b, n_steps, max_rel, F32_TOL, name)
+    assert max_rel(r.mod_prefix.double().cpu().numpy(), want["m0"]) < F32_TOL
 
 
 @pytest.mark.parametrize("name", ["toy", "small"])

@@ -16,7 +16,8 @@ import torch
 
 from oracle import qi21_oracle as O
 from qi21_synth import configs as C
-from tests._harness import oracle_model, max_rel, rel_l2
+from tests._harness import (BF16_TOL, F32_TOL, assert_item_matches, gpu_steps, max_rel, oracle_item,
+                            oracle_model, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,56 +35,41 @@ def _run(B, w, dtype, wts, shared, n_steps=2):
     r = Qi21Runner(w, dtype, host_weights=wts, shared_prefix=shared)
     pre1 = C.host_prefix_hidden(dataclasses.replace(w, batch=1))           # the one shared prefix
     pre = np.repeat(pre1, 1 if shared else w.batch, axis=0)
-    x = torch.from_numpy(C.host_noise(w).astype(np.float32)).cuda()
-    v = torch.empty_like(x)
-    r.set_prefix_row()
-    r.prefix_extract(torch.from_numpy(pre.astype(np.float32)).cuda())
-    vs = []
-    for k in range(n_steps):
-        r.set_target_row(w.sigmas[k])
-        r.cached_step(x, v)
-        vs.append(v.double().cpu().numpy())
-        r.euler(x, v, w.sigmas[k], w.sigmas[k + 1], x)
-    torch.cuda.synchronize()
-    r.check_device()
-    return vs, x.double().cpu().numpy(), r, pre1[0]
+    x0 = torch.from_numpy(C.host_noise(w).astype(np.float32)).cuda()
+    got = gpu_steps(r, torch.from_numpy(pre.astype(np.float32)).cuda(), x0, w.sigmas, n_steps)
+    return got, r, pre1[0]
 
 
 def _oracle(w, model, pre1, n_steps=2):
     seq = O.make_sequence(w.segments)
     x0 = C.host_noise(w)
-    return [O.run_image(model, seq, pre1, x0[b], w.sigmas[:n_steps + 1], use_cache=True) for b in range(w.batch)]
+    return [oracle_item(model, seq, pre1, x0[b], w.sigmas, n_steps) for b in range(w.batch)]
 
 
 @pytest.mark.parametrize("name", ["small", "small64"])
 def test_shared_prefix_f32_matches_oracle(B, name):
+    """Every request's v_theta, latent and per-layer target K/V, and the one
+    prefix copy's K/V of every layer, within 1e-4 max relative error."""
     w = dataclasses.replace(C.make_workload(name), batch=3)
     model, wts = oracle_model(w, "float32")
-    vs, x, r, pre1 = _run(B, w, B.QI21_DTYPE_F32, wts, shared=True)
+    got, r, pre1 = _run(B, w, B.QI21_DTYPE_F32, wts, shared=True)
     want = _oracle(w, model, pre1)
     for b in range(w.batch):
-        for k in range(2):
-            assert max_rel(vs[k][b], want[b]["velocities"][k]) < 1e-4
-        assert max_rel(x[b], want[b]["xs"][-1]) < 1e-4
-    K, V = r.cache_kv()
-    ck, cv = want[0]["cache_k"], want[0]["cache_v"]
-    assert max_rel(K[:, :r.P].double().cpu().numpy(), ck) < 1e-4
-    assert max_rel(V[:, :r.P].double().cpu().numpy(), cv) < 1e-4
+        assert_item_matches(got, want[b], b, 2, max_rel, F32_TOL, name)
 
 
 @pytest.mark.parametrize("name", ["small", "small64"])
 def test_shared_prefix_bf16_tensor_cores(B, name):
     w = dataclasses.replace(C.make_workload(name), batch=3)
     model, wts = oracle_model(w, "bfloat16")
-    vs, x, _, pre1 = _run(B, w, B.QI21_DTYPE_BF16, wts, shared=True)
+    got, _, pre1 = _run(B, w, B.QI21_DTYPE_BF16, wts, shared=True)
     want = _oracle(w, model, pre1)
     for b in range(w.batch):
-        for k in range(2):
-            assert rel_l2(vs[k][b], want[b]["velocities"][k]) < 2e-2
-        assert rel_l2(x[b], want[b]["xs"][-1]) < 2e-2
+        assert_item_matches(got, want[b], b, 2, rel_l2, BF16_TOL, name)
     # the per-item layout fed the same prefix three times computes the same steps
-    vs2, x2, _, _ = _run(B, w, B.QI21_DTYPE_BF16, wts, shared=False)
-    assert rel_l2(x, x2) < 1e-2
+    got2, _, _ = _run(B, w, B.QI21_DTYPE_BF16, wts, shared=False)
+    assert rel_l2(got["x"][-1], got2["x"][-1]) < 1e-2
+    assert rel_l2(got["tk"][-1], got2["tk"][-1]) < 1e-2
 
 
 def test_shared_prefix_whole_image_graph(B):
@@ -102,5 +88,5 @@ def test_shared_prefix_whole_image_graph(B):
     r.check_device()
     want = _oracle(w, model, pre1[0], n_steps=len(w.sigmas) - 1)
     for b in range(w.batch):
-        assert max_rel(x.double().cpu().numpy()[b], want[b]["xs"][-1]) < 1e-4
+        assert max_rel(x.double().cpu().numpy()[b], want[b]["x"][-1]) < F32_TOL
     del g

@@ -1,16 +1,23 @@
 """BF16 mode on the tcgen05 tensor-core kernels: parity with the fp64 oracle
-(2e-2 relative L2) and agreement with the CUDA-core kernel family on the same
-bf16 storage (same roundings up to accumulation order)."""
+(2e-2 relative L2) on every layer's prefix K/V, every layer's target K/V of
+each cached step, v_theta and the latent; and agreement with the CUDA-core
+kernel family on the same bf16 storage (same roundings up to accumulation
+order).
+
+The workloads use the parity weight recipe (O(1) modulation gates, an
+attention branch as large as the residual stream): replacing the attention by
+zeros moves every compared tensor by more than ten times the tolerance
+(tests/test_parity_strength.py), so these tests fail for a wrong attention.
+"""
 import numpy as np
 import pytest
 import torch
 
 from oracle import qi21_oracle as O
 from qi21_synth import configs as C
-from tests._harness import oracle_model, rel_l2
+from tests._harness import BF16_TOL, assert_item_matches, gpu_steps, oracle_item, oracle_model, rel_l2
 
 pytestmark = pytest.mark.gpu
-BF16_TOL = 2e-2
 
 
 @pytest.fixture(scope="module")
@@ -26,27 +33,18 @@ def _run(B, w, wts, tc: int, n_steps: int):
     B.qi21_set_tensor_cores(tc)
     try:
         r = Qi21Runner(w, B.QI21_DTYPE_BF16, host_weights=wts)
+        fam = B.qi21_kernel_family(r.cfg)
+        assert fam == (B.QI21_FAMILY_TENSOR_CORES if tc else B.QI21_FAMILY_CUDA_CORES)
         pre = torch.from_numpy(C.host_prefix_hidden(w).astype(np.float32)).cuda()
-        x = torch.from_numpy(C.host_noise(w).astype(np.float32)).cuda()
-        v = torch.empty_like(x)
-        r.set_prefix_row()
-        r.prefix_extract(pre)
-        vs, xs = [], []
-        for k in range(n_steps):
-            r.set_target_row(w.sigmas[k])
-            r.cached_step(x, v)
-            vs.append(v.double().cpu().numpy())
-            r.euler(x, v, w.sigmas[k], w.sigmas[k + 1], x)
-            xs.append(x.double().cpu().numpy())
+        x0 = torch.from_numpy(C.host_noise(w).astype(np.float32)).cuda()
+        got = gpu_steps(r, pre, x0, w.sigmas, n_steps)
+        vf = torch.empty_like(x0)
+        xl = torch.from_numpy(got["x"][-1].astype(np.float32)).cuda()
+        r.full_recompute(pre, xl, vf)
         torch.cuda.synchronize()
         r.check_device()
-        K, V = r.cache_kv()
-        kv = (K[:, :, :r.P].double().cpu().numpy(), V[:, :, :r.P].double().cpu().numpy())
-        vf = torch.empty_like(x)
-        r.full_recompute(pre, x, vf)
-        torch.cuda.synchronize()
-        r.check_device()
-        return vs, xs, kv, vf.double().cpu().numpy(), x.double().cpu().numpy(), r
+        got["vfull"] = vf.double().cpu().numpy()
+        return got
     finally:
         B.qi21_set_tensor_cores(1)
 
@@ -57,11 +55,12 @@ def test_tc_family_agrees_with_cuda_core_family(B, name):
     _, wts = oracle_model(w, "bfloat16")
     a = _run(B, w, wts, 1, 2)
     b = _run(B, w, wts, 0, 2)
-    assert rel_l2(a[2][0], b[2][0]) < 1e-2     # prefix K of every layer
-    assert rel_l2(a[2][1], b[2][1]) < 1e-2     # prefix V
+    for key in ("pk", "pv"):
+        assert rel_l2(a[key], b[key]) < 1e-2, key
     for k in range(2):
-        assert rel_l2(a[0][k], b[0][k]) < 1e-2
-    assert rel_l2(a[3], b[3]) < 1e-2           # full recompute
+        for key in ("tk", "tv", "v"):
+            assert rel_l2(a[key][k], b[key][k]) < 1e-2, f"{key} step {k}"
+    assert rel_l2(a["vfull"], b["vfull"]) < 1e-2
 
 
 @pytest.mark.parametrize("name", ["small", "small64", "small_t1"])
@@ -72,20 +71,11 @@ def test_tc_matches_oracle(B, name):
     pre = C.host_prefix_hidden(w)
     x0 = C.host_noise(w)
     n_steps = 3
-    vs, xs, (gk, gv), vfull, xlast, r = _run(B, w, wts, 1, n_steps)
-    m0, _ = O.modulation(0.0, model.wts, 4)
+    got = _run(B, w, wts, 1, n_steps)
     for b in range(w.batch):
-        ck, cv = O.prefix_extract(model, seq, pre[b], m0)
-        assert rel_l2(gk[:, b], ck) < BF16_TOL
-        assert rel_l2(gv[:, b], cv) < BF16_TOL
-        x = x0[b]
-        for k in range(n_steps):
-            mt, sf = O.modulation(1000.0 * w.sigmas[k], model.wts, 4)
-            v, _ = O.cached_step(model, seq, ck, cv, x, mt, sf)
-            x = O.euler_step(x, v, w.sigmas[k], w.sigmas[k + 1])
-            assert rel_l2(vs[k][b], v) < BF16_TOL, f"v step {k} item {b}"
-            assert rel_l2(xs[k][b], x) < BF16_TOL, f"x step {k} item {b}"
-        # full recompute at sigma_{n_steps} on the last latent
+        want = oracle_item(model, seq, pre[b], x0[b], w.sigmas, n_steps)
+        assert_item_matches(got, want, b, n_steps, rel_l2, BF16_TOL, name)
+        # full recompute at sigma_{n_steps - 1} on the last latent
         mt, sf = O.modulation(1000.0 * w.sigmas[n_steps - 1], model.wts, 4)
-        ref = O.joint_forward(model, seq, pre[b], xlast[b], m0, mt, sf)["v"]
-        assert rel_l2(vfull[b], ref) < BF16_TOL
+        ref = O.joint_forward(model, seq, pre[b], got["x"][-1][b], want["m0"], mt, sf)["v"]
+        assert rel_l2(got["vfull"][b], ref) < BF16_TOL
