@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="skip the whole-image CUDA-graph timing")
     ap.add_argument("--batched-requests", type=int, default=4,
                     help="requests sharing one prefix cache in the denoise-batching timing (0: skip)")
+    ap.add_argument("--configs", default="block,mid,large",
+                    help="other workloads timed in short runs beside the headline (comma list, '' to skip)")
     return ap.parse_args()
 
 
@@ -95,14 +97,49 @@ def kernel_bytes(w):
     }
 
 
+def _find_mhz(j, want_sustained):
+    """A clock (MHz) recorded beside the peaks: the first numeric field whose key
+    names a clock (mhz / clock) and, as asked, does or does not say sustained."""
+    stack = [("", j)]
+    while stack:
+        key, v = stack.pop(0)
+        if isinstance(v, dict):
+            stack += [((key + "." + k).lower(), x) for k, x in v.items()]
+            continue
+        if not isinstance(v, (int, float)) or isinstance(v, bool):
+            continue
+        if ("mhz" in key or "clock" in key) and "mem" not in key and "hbm" not in key and "max" not in key:
+            if ("sustain" in key) == want_sustained:
+                return float(v)
+    return None
+
+
 def load_peaks():
+    """Roofline denominators: the measured peaks when present, else the
+    pool's earlier measurement (burst 1.59 PF, sustained ~1.4 PF at ~1.3 GHz
+    under the power cap, copy 6.65 TB/s)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             j = json.load(f)
         return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
-                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "src": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "src": "measured",
+                "sustained_mhz": _find_mhz(j, True), "burst_mhz": _find_mhz(j, False)}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback",
+            "sustained_mhz": 1300.0, "burst_mhz": None}
+
+
+def tensor_fracs(tflops, peaks, run_mhz):
+    """A tensor-core rate against the peaks: the sustained figure (a kernel
+    timed inside a long step), the burst figure, and the clock-normalised ratio
+    (work per SM clock against the sustained peak's work per clock), which
+    cancels the difference between the run's clock and the peak's."""
+    out = {"frac_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+           "frac_burst": round(tflops / peaks["bf16_tflops"], 4)}
+    if run_mhz and peaks.get("sustained_mhz"):
+        out["frac_per_clock_vs_sustained"] = round(
+            (tflops / run_mhz) / (peaks["bf16_tflops_sustained"] / peaks["sustained_mhz"]), 4)
+    return out
 
 
 # The files a kernel's code and launch configuration come from: a stored ncu
@@ -189,17 +226,18 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
-# Target rows of the one-block oracle sample behind `cpu_baseline` (about 10-30 s of
-# host work at full width); the reference arm times 512-row samples per step so that
-# its warm-up + timed steps end within a few minutes.
-CPU_BASELINE_ROWS = 4096
-REFERENCE_ROWS = 512
+# Both the GPU arm's cpu_baseline and the reference arm time the same bounded
+# sample: one of the L blocks of the cached step at full width, for ORACLE_ROWS
+# target rows attending to all P + N keys (the other targets' K/V are synthetic
+# cache rows). Its time is extrapolated to a whole step (x L blocks x N / rows),
+# and that extrapolation is stated beside every figure derived from it.
+ORACLE_ROWS = 512
+SINGLE_THREAD_ROWS = 128
+CPU_BASELINE_SECONDS = 12.0
 
 
-def oracle_sample_inputs(w, rows=REFERENCE_ROWS, seed=4321):
-    """Inputs of the oracle timing sample: one block of the cached step at full
-    width for `rows` target tokens attending to all P + N keys (the other
-    targets' K/V are synthetic cache rows). Drawn once, reused by every timed run."""
+def oracle_sample_inputs(w, rows=ORACLE_ROWS, seed=4321):
+    """Inputs of the oracle timing sample. Drawn once, reused by every timed run."""
     from oracle import qi21_oracle as O
 
     rows = min(rows, w.n_target)
@@ -220,26 +258,181 @@ def oracle_sample_inputs(w, rows=REFERENCE_ROWS, seed=4321):
             "omega": O.rope_omega_axial(Dh), "allowed": np.ones((rows, extra + rows), dtype=bool)}
 
 
-def oracle_sample(w, rows=REFERENCE_ROWS, seed=4321, inputs=None):
-    """Time the fp64 oracle on the bounded sample of oracle_sample_inputs. Returns
-    (seconds, target tokens/s scaled to all L blocks, threads, description)."""
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, inputs, threads=None):
+    """Seconds of one run of the fp64 oracle's block on the sample (all BLAS
+    threads, or `threads` of them)."""
     from oracle import qi21_oracle as O
 
     sh = w.shape
-    x = inputs if inputs is not None else oracle_sample_inputs(w, rows, seed)
+    x = inputs
+
+    def run():
+        t0 = time.perf_counter()
+        O.dit_block(x["h"], x["mods"], x["lw"], sh.n_heads, x["coords"], x["omega"], (x["kc"], x["vc"]),
+                    x["allowed"], sh.ln_eps, sh.qk_eps)
+        return time.perf_counter() - t0
+
+    if threads is None:
+        return run()
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        return run()
+
+
+def oracle_tokens_per_s(w, rows, seconds):
+    """Target tokens/s of a whole cached step extrapolated from one block's sample."""
+    return rows / (seconds * w.shape.n_layers)
+
+
+def oracle_desc(w, rows, threads):
+    return (f"one of {w.shape.n_layers} blocks of the cached step at d={w.shape.d_model}, {rows} target rows "
+            f"attending to {w.n_prefix + w.n_target} keys, fp64 numpy on {threads} threads")
+
+
+def extrapolation(w, rows):
+    return f"x{w.shape.n_layers} blocks x {w.n_target}/{rows} rows (one block of a {rows}-row sample timed)"
+
+
+def cpu_baseline(w):
+    """The oracle on the host cores, timed on the shared sample repeated for
+    about CPU_BASELINE_SECONDS, plus a single-thread timing on a smaller sample."""
+    x = oracle_sample_inputs(w)
+    threads = _blas_threads()
+    times = []
+    t_end = time.perf_counter() + CPU_BASELINE_SECONDS
+    while not times or (time.perf_counter() < t_end and len(times) < 50):
+        times.append(oracle_sample(w, x))
+    sec = statistics.mean(times)
+    out = {"value": round(oracle_tokens_per_s(w, x["rows"], sec), 4), "unit": UNIT, "cores": threads,
+           "kind": "oracle", "sample": oracle_desc(w, x["rows"], threads),
+           "sample_seconds": round(sec, 3), "sample_reps": len(times),
+           "extrapolated": extrapolation(w, x["rows"])}
     try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    O.dit_block(x["h"], x["mods"], x["lw"], sh.n_heads, x["coords"], x["omega"], (x["kc"], x["vc"]), x["allowed"],
-                sh.ln_eps, sh.qk_eps)
-    dt = time.perf_counter() - t0
-    tok_s = x["rows"] / (dt * sh.n_layers)
-    desc = (f"one of {sh.n_layers} blocks of the cached step at d={sh.d_model}, {x['rows']} target rows attending "
-            f"to {w.n_prefix + w.n_target} keys, fp64 numpy; time x {sh.n_layers} blocks per token")
-    return dt, tok_s, threads, desc
+        x1 = oracle_sample_inputs(w, rows=SINGLE_THREAD_ROWS)
+        s1 = oracle_sample(w, x1, threads=1)
+        out["single_thread"] = {"value": round(oracle_tokens_per_s(w, x1["rows"], s1), 4), "unit": UNIT,
+                                "cores": 1, "sample_seconds": round(s1, 3),
+                                "sample": oracle_desc(w, x1["rows"], 1),
+                                "extrapolated": extrapolation(w, x1["rows"])}
+    except Exception as e:   # threadpoolctl missing: report why
+        out["single_thread"] = {"unavailable": str(e)}
+    return out
+
+
+def kernel_table(prof, kf, kb, peaks, run_mhz):
+    """Per-kernel launches, time, share of the step and achieved rate against
+    its roofline (tensor-core kernels: TFLOP/s; memory-bound ones: GB/s of
+    algorithmic bytes against the measured copy bandwidth)."""
+    total = sum(t for _, t in prof.values()) or 1.0
+    kernels = {}
+    for name, (n, tot) in prof.items():
+        avg = tot / n
+        ent = {"launches": n, "total_ms": round(tot, 3), "avg_ms": round(avg, 4), "share": round(tot / total, 4)}
+        if name in kf:
+            ach = kf[name] / (avg / 1e3) / 1e12
+            ent["tflops"] = round(ach, 1)
+            ent.update(tensor_fracs(ach, peaks, run_mhz))
+        elif name in kb:
+            ach = kb[name] / (avg / 1e3) / 1e9
+            ent.update({"gbs": round(ach, 1), "frac_hbm": round(ach / peaks["hbm_gbs"], 3)})
+        kernels[name] = ent
+    return kernels
+
+
+def time_config(cname, r_main, w_main, dev, world, rank):
+    """Short run of another workload beside the headline: extract once, then
+    a few cached steps (modulation + cached step + Euler) timed with CUDA events
+    as the max over ranks, with per-kernel times and the SM clocks sampled.
+    A workload of the headline's model shape reuses its device weights."""
+    import dataclasses
+
+    import torch
+    from prefix_kv_cached_b200 import binding as B
+    from prefix_kv_cached_b200.runner import Qi21Runner
+    from qi21_synth import configs as C
+    from qi21_synth.gen import normal_torch
+
+    wc = C.make_workload(cname)
+    wc = dataclasses.replace(wc, seed=wc.seed + 1000 * rank)
+    if wc.shape == w_main.shape:
+        rc = Qi21Runner(wc, B.QI21_DTYPE_BF16, device=str(dev), share_weights_with=r_main)
+    else:
+        rc = Qi21Runner(wc, B.QI21_DTYPE_BF16, device=str(dev), weights=C.device_weights(wc, torch.bfloat16, dev))
+    sh = wc.shape
+    pre = normal_torch(wc.seed, "prefix_hidden", (wc.batch, wc.n_prefix, sh.d_model), device=dev,
+                       dtype=torch.float32)
+    x = normal_torch(wc.seed, "noise", (wc.batch, wc.n_target, sh.latent_ch), device=dev, dtype=torch.float32)
+    v = torch.empty_like(x)
+    st = torch.cuda.current_stream(dev)
+    sig = wc.sigmas
+    rc.set_prefix_row()
+    rc.prefix_extract(pre)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    rc.prefix_extract(pre)
+    e1.record(st)
+    torch.cuda.synchronize()
+    extract_ms = dist_max(e0.elapsed_time(e1), world)
+
+    def step(k):
+        i = k % (len(sig) - 1)
+        rc.set_target_row(sig[i])
+        rc.cached_step(x, v)
+        rc.euler(x, v, sig[i], sig[i + 1], x)
+
+    steps = 4 if wc.n_target * wc.batch > 8192 else 20
+    warm = 3
+    for k in range(warm):
+        step(k)
+    torch.cuda.synchronize()
+    rc.check_device()
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    B.qi21_profile_reset()
+    B.qi21_profile_enable(1)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(st)
+    for k in range(steps):
+        step(k)
+    t1.record(st)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    clk = clocks.stop()
+    B.qi21_profile_enable(0)
+    prof = B.qi21_profile_read()
+    ms = dist_max(t0.elapsed_time(t1), world) / steps
+    rc.check_device()
+    del rc, pre, x, v
+    torch.cuda.empty_cache()
+    return {"w": wc, "ms": ms, "extract_ms": extract_ms, "steps": steps, "warmup": warm, "clocks": clk,
+            "prof": prof}
+
+
+def config_record(res, world, peaks):
+    """JSON sub-record of a time_config() result."""
+    wc, ms, clk = res["w"], res["ms"], res["clocks"]
+    tokens = wc.batch * wc.n_target
+    tflops = step_flops(wc) / (ms / 1e3) / 1e12
+    fr = tensor_fracs(tflops, peaks, clk.get("sm_mhz"))
+    return {"workload": config_dict(wc)["workload"], "ms_per_step": round(ms, 3),
+            "target_tokens_per_s": round(world * tokens / (ms / 1e3), 1), "step_tflops": round(tflops, 1),
+            "tensor_frac_step": fr["frac_sustained"], "tensor_frac_step_burst": fr["frac_burst"],
+            "tensor_frac_step_per_clock": fr.get("frac_per_clock_vs_sustained"),
+            "extract_ms": round(res["extract_ms"], 3), "steps": res["steps"], "warmup": res["warmup"],
+            "clocks": clk, "kernels": kernel_table(res["prof"], kernel_flops(wc), kernel_bytes(wc), peaks,
+                                                   clk.get("sm_mhz"))}
 
 
 # ----------------------------------------------------------------------------- distributed helpers
@@ -290,24 +483,31 @@ def dist_done(world: int):
 
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, w, world, rank):
+    """The reference arm: the fp64 oracle as it stands (the pages publish no
+    code), one bounded sample per step (see ORACLE_ROWS), on rank 0 only."""
     if rank != 0:
         return 0
-    steps = []
-    desc = threads = None
     inputs = oracle_sample_inputs(w)
+    threads = _blas_threads()
+    steps = []
     for i in range(args.warmup + args.steps):
-        dt, tok_s, threads, desc = oracle_sample(w, inputs=inputs)
+        dt = oracle_sample(w, inputs)
         if i >= args.warmup:
             steps.append(dt)
-    dt = statistics.mean(steps)
-    rows = min(REFERENCE_ROWS, w.n_target)
-    tok_s = rows / (dt * w.shape.n_layers)
+    sec = statistics.mean(steps)
+    rows = inputs["rows"]
+    tok_s = oracle_tokens_per_s(w, rows, sec)
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 * w.shape.n_layers * w.n_target / rows,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3 * w.shape.n_layers * w.n_target / rows,
+        "ms_per_step_how": "extrapolated: " + extrapolation(w, rows),
+        "sample_seconds": round(sec, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(w),
-        "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": oracle_desc(w, rows, threads), "sample_seconds": round(sec, 4),
+                         "extrapolated": extrapolation(w, rows)},
         "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -507,40 +707,44 @@ def main():
         e2e = {"value": world * tokens * args.steps / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e_ms / args.steps}
 
+    # other workloads, short runs beside the headline (the same model's weights where the shape matches)
+    other_raw = {}
+    for cname in [c.strip() for c in args.configs.split(",") if c.strip()]:
+        if cname != args.workload:
+            other_raw[cname] = time_config(cname, r, w, dev, world, rank)
+
     if rank == 0:
         peaks = load_peaks()
+        other_configs = {k: config_record(v, world, peaks) for k, v in other_raw.items()} or None
         kf = kernel_flops(w)
         kb = kernel_bytes(w)
         kernels = {}
-        for name, (n, tot) in prof.items():
-            avg = tot / n
-            ent = {"launches": n, "total_ms": round(tot, 3), "avg_ms": round(avg, 4),
-                   "share": round(tot / sum(t for _, t in prof.values()), 4)}
-            if name in kf:
-                ach = kf[name] / (avg / 1e3) / 1e12
-                ent.update({"tflops": round(ach, 1), "frac_sustained": round(ach / peaks["bf16_tflops_sustained"], 3)})
-            elif name in kb:
-                ach = kb[name] / (avg / 1e3) / 1e9
-                ent.update({"gbs": round(ach, 1), "frac_hbm": round(ach / peaks["hbm_gbs"], 3)})
-            kernels[name] = ent
+        kernels = kernel_table(prof, kf, kb, peaks, clk.get("sm_mhz"))
         dom = max(((k, e) for k, e in kernels.items() if k in kf), key=lambda t: t[1]["total_ms"], default=None)
         roof = None
         if dom:
             name, ent = dom
             ach = kf[name] / (ent["avg_ms"] / 1e3) / 1e12
+            fr = tensor_fracs(ach, peaks, clk.get("sm_mhz"))
             roof = {"kernel": name, "bound": "tensor", "achieved": round(ach, 1),
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                    "frac": round(ach / peaks["bf16_tflops_sustained"], 4), "traffic": load_traffic(name),
+                    "frac": fr["frac_sustained"], "traffic": load_traffic(name),
                     "peak_src": f"{peaks['src']} bf16 sustained (kernel timed inside a long step)",
+                    "frac_burst": fr["frac_burst"], "peak_burst": peaks["bf16_tflops"],
+                    "frac_per_clock_vs_sustained": fr.get("frac_per_clock_vs_sustained"),
+                    "peak_sustained_mhz": peaks.get("sustained_mhz"), "run_sm_mhz": clk.get("sm_mhz"),
                     "algorithmic_flops_per_launch": kf[name]}
         sflops = step_flops(w)
         step_tflops = sflops / (ms_step / 1e3) / 1e12
+        step_fr = tensor_fracs(step_tflops, peaks, clk.get("sm_mhz"))
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded SplitMix64/Box-Muller draws)",
             "config": config_dict(w),
-            "tensor_frac_step": round(step_tflops / peaks["bf16_tflops_sustained"], 4),
+            "tensor_frac_step": step_fr["frac_sustained"],
+            "tensor_frac_step_burst": step_fr["frac_burst"],
+            "tensor_frac_step_per_clock": step_fr.get("frac_per_clock_vs_sustained"),
             "step_tflops": round(step_tflops, 1),
             "step_ms_percentiles": pct,
             "batched_shared_prefix": batched,
@@ -548,11 +752,10 @@ def main():
                           "tokens_per_s": round(world * tokens / ((extract_ms + 8 * ms_step) / 1e3), 1),
                           "graph": image},
             "roofline": roof, "kernels": kernels, "gpu_launches": launches[0], "clocks": clk, "e2e": e2e,
+            "configs": other_configs,
         }
         if world == 1 and not args.no_cpu_baseline:
-            dt, tok_s, threads, desc = oracle_sample(w, rows=CPU_BASELINE_ROWS)
-            line["cpu_baseline"] = {"value": round(tok_s, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": desc, "seconds": round(dt, 2)}
+            line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
     dist_done(world)
     return 0

@@ -249,9 +249,10 @@ qi21_status qi21_modulation_sigma(const qi21_config *cfg, const qi21_weights *w,
  * another allocator, or they must never call cudaMalloc because it can block).
  * Same result as qi21_modulation, but takes no workspace: its two
  * timestep-MLP intermediate vectors live in a fixed file-scope device array of
- * 2 * QI21_NOALLOC_MAX_D floats instead. Returns QI21_ERR_UNSUPPORTED when
- * d_model > QI21_NOALLOC_MAX_D (or time_dim > 512), before anything is
- * enqueued. Allocates nothing and calls no allocating routine. The first call
+ * 2 * QI21_NOALLOC_MAX_D floats instead. Applies the shape checks of
+ * qi21_modulation and returns QI21_ERR_UNSUPPORTED when d_model >
+ * QI21_NOALLOC_MAX_D, before anything is enqueued; a failed launch returns
+ * QI21_ERR_CUDA. Allocates nothing and calls no allocating routine. The first call
  * on a device looks up that device's address of the array
  * (cudaGetSymbolAddress, with the device current), so make that first call
  * before any stream capture. Every call on a device shares the one array and

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 #include <type_traits>
@@ -77,6 +78,24 @@ struct Launcher {
 
 static inline bool al16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
 
+// The dynamic shared-memory opt-in above 48 KB is a per-device attribute of a
+// kernel: each call site keeps one flag per device and sets it on the current
+// device the first time (the call is not a stream operation, so this also
+// works while a stream is being captured).
+constexpr int kMaxDevices = 64;
+using DeviceFlags = std::atomic<int>[kMaxDevices];
+
+template <typename K>
+static void smem_opt_in(K *kernel, int bytes, DeviceFlags &done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return;   // the launch reports the error
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire) >= bytes) return;
+    if (cudaFuncSetAttribute((const void *)kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+            cudaSuccess &&
+        dev >= 0 && dev < kMaxDevices)
+        done[dev].store(bytes, std::memory_order_release);
+}
+
 static inline int grid_for(int64_t n, int threads, int cap = 148 * 16) {
     int64_t g = (n + threads - 1) / threads;
     if (g < 1) g = 1;
@@ -120,13 +139,14 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t 
 }
 
 static int num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
+    static std::atomic<int> count[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && count[dev].load() > 0) return count[dev].load();
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    if (dev >= 0 && dev < kMaxDevices) count[dev].store(n);
     return n;
 }
 
@@ -134,11 +154,8 @@ template <int EPI>
 static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, const CUtensorMap &b0,
                            const CUtensorMap &b1, const CUtensorMap &b2, const GemmParams &p) {
     constexpr size_t smem = tc_smem_bytes<EPI>();
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(k_gemm_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        attr = true;
-    }
+    static DeviceFlags attr;
+    smem_opt_in(k_gemm_tc<EPI>, (int)smem, attr);
     const int tiles = p.m_blocks * p.n_blocks * p.ksplit;
     const int grid = tiles < num_sms() ? tiles : num_sms();
     L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
@@ -176,11 +193,8 @@ template <int DH>
 static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                            const AttnParams &p, int B) {
     using Cf = AttnCfg<DH>;
-    static bool attr = false;
-    if (!attr) {
-        cudaFuncSetAttribute(k_attn_tc<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
-        attr = true;
-    }
+    static DeviceFlags attr;
+    smem_opt_in(k_attn_tc<DH>, (int)Cf::SMEM, attr);
     dim3 grid((p.Mq + Cf::BQ - 1) / Cf::BQ, p.H, B);
     L.run("attn", [&] { k_attn_tc<DH><<<grid, Cf::THREADS, Cf::SMEM, L.st>>>(q, k, v, p); });
 }
@@ -391,11 +405,8 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
                 launch_attn_tc<64>(L, maps.q4, maps.k4, maps.v4, ap, a.B);
         } else {
             const size_t smem = sizeof(float) * (3 * 32 * (Dh + 1) + 32 * 33);
-            static bool attr_set = false;
-            if (!attr_set) {
-                cudaFuncSetAttribute(k_attn_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-                attr_set = true;
-            }
+            static DeviceFlags attr;
+            smem_opt_in(k_attn_simt<T>, 64 * 1024, attr);
             dim3 grid((a.M + 31) / 32, H, a.B);
             L.run("attn_simt", [&] {
                 if (a.shared)
@@ -477,11 +488,8 @@ static void launch_final(Launcher &L, const qi21_config &c, const float *h, int 
         return;
     }
     const size_t smem = sizeof(float) * 4 * d;
-    static bool attr_set[2] = {false, false};
-    if (smem > 48 * 1024 && !attr_set[sizeof(T) == 2]) {
-        cudaFuncSetAttribute(k_final<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        attr_set[sizeof(T) == 2] = true;
-    }
+    static DeviceFlags attr;
+    if (smem > 48 * 1024) smem_opt_in(k_final<T>, 200 * 1024, attr);
     L.run("final", [&] {
         k_final<T><<<(rows + 3) / 4, 256, smem, L.st>>>(h, M, off, N, d, sf, (const T *)w_out, c.latent_ch, c.ln_eps,
                                                        v, rows);
@@ -512,6 +520,8 @@ static qi21_status check_shapes(const qi21_config *c) {
     if (c->dtype == QI21_DTYPE_BF16 && tc_enabled() && !tc_supported(*c)) return QI21_ERR_UNSUPPORTED;
     return QI21_OK;
 }
+
+qi21_status check_config_shapes(const qi21_config *c) { return check_shapes(c); }
 
 static qi21_status finish(Launcher &L) { return L.status; }
 
@@ -544,11 +554,8 @@ static qi21_status modulation_impl(const qi21_config *c, const qi21_weights *w, 
     const size_t xs = sizeof(float) * d;
     auto run = [&](auto *wt) {
         using T = std::remove_const_t<std::remove_pointer_t<decltype(wt)>>;
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(k_gemv2<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-            attr = true;
-        }
+        static DeviceFlags attr;
+        smem_opt_in(k_gemv2<T>, 64 * 1024, attr);
         if (emb)
             L.run("temb_in", [&] { k_temb_in<T><<<(d + 7) / 8, 256, 0, st>>>((const T *)w->w_t1, *emb, K0, d, a1); });
         else

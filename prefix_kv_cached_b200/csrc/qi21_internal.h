@@ -31,6 +31,10 @@ inline size_t dtype_bytes(int32_t dtype) { return dtype == QI21_DTYPE_BF16 ? 2 :
 // Kernel family of the BF16 mode (process-wide; qi21_set_tensor_cores).
 bool tc_enabled();
 
+// The shape checks every device entry point applies before enqueueing work:
+// QI21_ERR_INVALID_ARG / SHAPE / UNSUPPORTED, or QI21_OK.
+qi21_status check_config_shapes(const qi21_config *c);
+
 // Packed weight buffer of qi21_pack_weights: the 15 tensors of qi21_weights in
 // struct order, [out][in] (stacked [L][out][in]), each on a 256-byte boundary.
 struct PackedLayout {

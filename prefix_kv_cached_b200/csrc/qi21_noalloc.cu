@@ -18,8 +18,6 @@
 #include "qi21_internal.h"
 #include "qi21_simt.cuh"
 
-bool qi21_config_ok(const qi21_config *c);
-
 namespace qi21 {
 
 // [0, d): silu(w_t1 . emb(t));  [d, 2d): e = w_t2 . (first half).
@@ -55,9 +53,10 @@ using namespace qi21;
 extern "C" qi21_status qi21_modulation_noalloc(const qi21_config *c, const qi21_weights *w, double t,
                                                float *mod_row, float *scale_final, void *stream) {
     if (!c || !w) return QI21_ERR_INVALID_ARG;
-    if (!qi21_config_ok(c)) return QI21_ERR_SHAPE;
+    // the same shape checks as qi21_modulation, then this entry point's own limit
+    const qi21_status shape = check_config_shapes(c);
+    if (shape != QI21_OK) return shape;
     if (c->d_model > QI21_NOALLOC_MAX_D) return QI21_ERR_UNSUPPORTED;   // scratch holds 2 * QI21_NOALLOC_MAX_D floats
-    if (c->time_dim > 512) return QI21_ERR_UNSUPPORTED;
     if (!aligned16(w->w_t1) || !aligned16(w->w_t2) || !aligned16(w->w_mod) || !aligned16(w->w_fin) ||
         !aligned16(mod_row) || !aligned16(scale_final))
         return QI21_ERR_INVALID_ARG;
@@ -70,18 +69,26 @@ extern "C" qi21_status qi21_modulation_noalloc(const qi21_config *c, const qi21_
     qi21_timestep_embedding(t, K0, emb.v);
     float *a1 = scratch, *e = scratch + d;
     const size_t xs = sizeof(float) * d;     // <= 32 KB: no opt-in above the 48 KB default needed
+    // each launch's own status is read right after it, as the other entry points do
+    auto launched = [] { return cudaGetLastError() == cudaSuccess; };
     if (c->dtype == QI21_DTYPE_BF16) {
         k_temb_in<bf16><<<(d + 7) / 8, 256, 0, st>>>((const bf16 *)w->w_t1, emb, K0, d, a1);
+        if (!launched()) return QI21_ERR_CUDA;
         k_gemv2<bf16><<<(d + 7) / 8, 256, xs, st>>>((const bf16 *)w->w_t2, d, e, (const bf16 *)w->w_t2, 0, e, a1,
                                                      d, 0);
+        if (!launched()) return QI21_ERR_CUDA;
         k_gemv2<bf16><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const bf16 *)w->w_mod, nch * d, mod_row,
                                                               (const bf16 *)w->w_fin, d, scale_final, e, d, 1);
+        if (!launched()) return QI21_ERR_CUDA;
     } else {
         k_temb_in<float><<<(d + 7) / 8, 256, 0, st>>>((const float *)w->w_t1, emb, K0, d, a1);
+        if (!launched()) return QI21_ERR_CUDA;
         k_gemv2<float><<<(d + 7) / 8, 256, xs, st>>>((const float *)w->w_t2, d, e, (const float *)w->w_t2, 0, e,
                                                       a1, d, 0);
+        if (!launched()) return QI21_ERR_CUDA;
         k_gemv2<float><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const float *)w->w_mod, nch * d, mod_row,
                                                                (const float *)w->w_fin, d, scale_final, e, d, 1);
+        if (!launched()) return QI21_ERR_CUDA;
     }
-    return cudaGetLastError() == cudaSuccess ? QI21_OK : QI21_ERR_CUDA;
+    return QI21_OK;
 }

@@ -255,3 +255,17 @@ def test_bf16_shape_without_tensor_core_kernels_is_refused(B):
 
 def test_lab_rope_omega_matches_oracle(B):
     assert np.array_equal(B.qi21_rope_omega_lab(), O.rope_omega_lab())
+
+
+def test_noalloc_applies_the_modulation_shape_checks(B):
+    """qi21_modulation_noalloc refuses what qi21_modulation refuses (here a BF16
+    head_dim the tensor-core kernels do not cover), before any launch."""
+    from prefix_kv_cached_b200.runner import make_config
+    cfg = make_config(C.ModelShape(256, 8, 32, 1, 768, 64, 256), B.QI21_DTYPE_BF16)
+    fake = 0x10000
+    w = B.qi21_weights(*([fake] * 15))
+    assert B.qi21_modulation(cfg, w, 500.0, fake, fake, fake, 1 << 30, 0) == B.QI21_ERR_UNSUPPORTED
+    assert B.qi21_modulation_noalloc(cfg, w, 500.0, fake, fake, 0) == B.QI21_ERR_UNSUPPORTED
+    bad = make_config(C.SMALL, B.QI21_DTYPE_F32)
+    bad.n_heads = 3
+    assert B.qi21_modulation_noalloc(bad, w, 500.0, fake, fake, 0) == B.QI21_ERR_SHAPE

@@ -8,7 +8,13 @@ row (two timesteps, so the second call overwrites what the first left in the
 shared array) and checks each result against qi21_modulation, which uses a
 caller workspace, within the fp32 tolerance of the parity tests (1e-4 max
 relative error). It also checks that a model wider than the array's limit is
-refused before anything runs. This file is collected last on purpose.
+refused before anything runs.
+
+The tests do not depend on test order: each builds its own runner and reads
+only what its own calls wrote (both calls of the array are fully written before
+they are read), so they pass alone in a fresh process and after every other
+test. The file name makes pytest collect it last only so that, should it fail,
+a run that stops at the first failure has already run every other test.
 """
 import numpy as np
 import pytest
