@@ -85,10 +85,15 @@ def kernel_bytes(w):
     sh = w.shape
     d, C = sh.d_model, sh.latent_ch
     R = w.batch * w.n_target
+    mb = -(-R // 128)
+    ks = max(1, min(8, d // 64, 148 // mb))   # K slices of the tensor-core final kernel
     return {
         "modln": R * d * (4 + 2),            # read fp32 h, write bf16
-        "img_in": R * C * 4 + R * d * 4,     # read x, write fp32 h
-        "final": R * d * 4 + R * C * 4,      # read h, write v
+        "img_in": R * C * 4 + R * d * 4,     # read x, write fp32 h (the GEMM launch reads x as bf16)
+        "img_in_cvt": R * C * (4 + 2),       # x to bf16 for the tensor-core img_in
+        "final": R * d * 4 + R * C * 4,      # read h, write v (the main launch of the final AdaLN + proj_out)
+        "final_prep": C * d * 2 * 2 + d * 4,  # W_out scaled by (1 + scale_final): read and write, read the scale
+        "final_reduce": ks * R * 68 * 4 + R * C * 4,   # the K-slice partials in, v out
         "euler": R * C * 12,
         # modulation: the two GEMV launches of a step read w_t2 (d x d) and then w_mod + w_fin
         # ((chunks + 1) d x d), bf16; bytes per launch = their mean

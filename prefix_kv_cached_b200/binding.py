@@ -12,7 +12,8 @@ import ctypes as ct
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqi21.so")
+# QI21_LIB selects another build of the library (the --debug build of build.py)
+LIB_PATH = os.environ.get("QI21_LIB") or os.path.join(_HERE, "libqi21.so")
 
 QI21_OK = 0
 QI21_ERR_INVALID_ARG = 1

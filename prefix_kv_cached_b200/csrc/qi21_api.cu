@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdio>
@@ -18,6 +19,7 @@
 #include "qi21_simt.cuh"
 #include "qi21_gemm_tc.cuh"
 #include "qi21_attn_tc.cuh"
+#include "qi21_final_tc.cuh"
 
 bool qi21_config_ok(const qi21_config *c);
 
@@ -59,7 +61,9 @@ struct Launcher {
             b = prof_event();
         }
         if (a) cudaEventRecord(a, st);
+        nvtxRangePushA(name);     // one NVTX range per launch, named as in qi21_profile_read
         f();
+        nvtxRangePop();
         ++count;
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) {
@@ -67,6 +71,19 @@ struct Launcher {
             status = QI21_ERR_CUDA;
             return;
         }
+#ifdef QI21_DEBUG
+        // debug build: wait for every kernel and name the one that failed (not
+        // while the stream is being captured, where synchronising is illegal)
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cap) == cudaSuccess && cap == cudaStreamCaptureStatusNone) {
+            e = cudaStreamSynchronize(st);
+            if (e != cudaSuccess) {
+                fprintf(stderr, "qi21: kernel %s failed: %s\n", name, cudaGetErrorString(e));
+                status = QI21_ERR_CUDA;
+                return;
+            }
+        }
+#endif
         if (b) {
             cudaEventRecord(b, st);
             std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -156,8 +173,8 @@ static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, 
     constexpr size_t smem = tc_smem_bytes<EPI>();
     static DeviceFlags attr;
     smem_opt_in(k_gemm_tc<EPI>, (int)smem, attr);
-    const int tiles = p.m_blocks * p.n_blocks * p.ksplit;
-    const int grid = tiles < num_sms() ? tiles : num_sms();
+    const int units = p.m_blocks * p.n_blocks * p.ksplit;
+    const int grid = (units < num_sms() && p.sk_tiles == 0) ? units : num_sms();
     L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
 }
 
@@ -172,6 +189,23 @@ static bool make_map_f32(CUtensorMap *m, const void *base, uint64_t inner, uint6
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 2-D tensor map [rows][inner] of bf16 or fp32 with a box of box_inner x
+// box_rows elements, 128-byte swizzle, zero fill outside the tensor.
+static bool make_map2d(CUtensorMap *m, const void *base, bool f32, uint64_t inner, uint64_t rows,
+                       uint32_t box_inner, uint32_t box_rows) {
+    if (!get_encode()) return false;
+    const uint64_t eb = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * eb};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -205,14 +239,13 @@ static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap 
 // rows: gate/up -15 %, down -11 %, QKV -7 %; at 4096 rows banding cost gate/up 3 %).
 static int gemm_group_m(int m_blocks) { return m_blocks > 32 ? 16 : 0; }
 
-// K slices for a residual GEMM: enough work units for about six waves of the
-// persistent grid (the reduce-add epilogue sums the slices in L2), at least
-// eight K blocks per slice.
-static int residual_ksplit(int tiles, int kblocks) {
-    const int target = 6 * num_sms();
-    int ks = 1;
-    while (ks < 4 && tiles * ks < target && kblocks / (ks + 1) >= 8) ++ks;
-    return ks;
+// Residual GEMMs (the reduce-add epilogue sums partial products in L2): whole
+// tiles for the full waves of the persistent grid, and the tiles of the last,
+// partial wave shared stream-K style, so that every CTA gets the same number of
+// K blocks and only about one extra partial tile per CTA is reduce-added.
+static int residual_sk_tiles(int tiles) {
+    const int g = num_sms();
+    return tiles % g;
 }
 
 struct TcMaps {
@@ -266,9 +299,25 @@ static void launch_modln(Launcher &L, const qi21_config &c, const float *h, T *o
     const int d = c.d_model;
     if (d % 4 == 0 && d <= 4 * 256 * 8) {
         const int vpt = (d / 4 + 255) / 256;
+        // as many blocks as fit on the GPU at once (each loops over rows)
+        auto grid_of = [&](auto kernel) {
+            static std::atomic<int> occ[kMaxDevices];
+            int dev = 0;
+            cudaGetDevice(&dev);
+            int per_sm = (dev >= 0 && dev < kMaxDevices) ? occ[dev].load() : 0;
+            if (per_sm <= 0) {
+                if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess ||
+                    per_sm <= 0)
+                    per_sm = 1;
+                if (dev >= 0 && dev < kMaxDevices) occ[dev].store(per_sm);
+            }
+            const int64_t g = (int64_t)per_sm * num_sms();
+            return (int)(rows < g ? rows : g);
+        };
         L.run("modln", [&] {
-#define QI21_LN(V)                                                                                           \
-    k_modln_vec<T, V><<<rows, 256, 0, L.st>>>(h, out, d, M, split, sc_lo, sc_hi, sh_lo, sh_hi, c.ln_eps)
+#define QI21_LN(V)                                                                                                \
+    k_modln_vec<T, V><<<grid_of(k_modln_vec<T, V>), 256, 0, L.st>>>(h, out, d, rows, M, split, sc_lo, sc_hi, sh_lo, \
+                                                                   sh_hi, c.ln_eps)
             if (vpt <= 1) QI21_LN(1);
             else if (vpt <= 2) QI21_LN(2);
             else if (vpt <= 4) QI21_LN(4);
@@ -422,7 +471,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             GemmParams g = gp;
             g.K = d;
             g.n_blocks = d / TC_BN;
-            g.ksplit = residual_ksplit(g.m_blocks * g.n_blocks, d / TC_BK);
+            g.sk_tiles = residual_sk_tiles(g.m_blocks * g.n_blocks);
             g.g_lo = tg1_lo;
             g.g_hi = tg1_hi;
             launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.h32, g);
@@ -442,7 +491,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             GemmParams g2 = gp;
             g2.K = F;
             g2.n_blocks = d / TC_BN;
-            g2.ksplit = residual_ksplit(g2.m_blocks * g2.n_blocks, F / TC_BK);
+            g2.sk_tiles = residual_sk_tiles(g2.m_blocks * g2.n_blocks);
             g2.g_lo = tg2_lo;
             g2.g_hi = tg2_hi;
             launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.h32, g2);
@@ -459,6 +508,73 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             });
         }
     }
+}
+
+// Tensor-core forms of img_in and of the final AdaLN + proj_out for the BF16
+// cached step (target rows contiguous in h): 64 latent channels, d a multiple
+// of 256 (every shape tc_supported() accepts).
+static bool tc_head_supported(const qi21_config &c) {
+    return c.dtype == QI21_DTYPE_BF16 && tc_enabled() && tc_supported(c) && c.latent_ch == 64;
+}
+
+static __global__ void k_to_bf16(const float *__restrict__ x, bf16 *__restrict__ y, int64_t n4) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 f = reinterpret_cast<const float4 *>(x)[i];
+        reinterpret_cast<uint2 *>(y)[i] = make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
+    }
+}
+
+// h[r][:] = x[r][:] W_img_in^T for rows [0, rows): the latent rounded to bf16,
+// then the tcgen05 GEMM with K = 64 whose epilogue stores fp32 rows of h.
+static void launch_img_in_tc(Launcher &L, const qi21_config &c, const float *x, const void *w_img_in, float *h,
+                             int rows, bf16 *xin, uint32_t *err) {
+    const int d = c.d_model, C = c.latent_ch;
+    const int64_t n4 = (int64_t)rows * C / 4;
+    L.run("img_in_cvt", [&] { k_to_bf16<<<grid_for(n4, 256), 256, 0, L.st>>>(x, xin, n4); });
+    CUtensorMap ma, mb, mh;
+    if (!make_map(&ma, xin, C, rows, 1, 128) || !make_map(&mb, w_img_in, C, d, 1, 128) ||
+        !make_map_f32(&mh, h, d, rows)) {
+        L.status = QI21_ERR_CUDA;
+        return;
+    }
+    GemmParams g{};
+    g.R = rows;
+    g.K = C;
+    g.m_blocks = (rows + TC_BM - 1) / TC_BM;
+    g.n_blocks = d / TC_BN;
+    g.ksplit = 1;
+    g.group_m = gemm_group_m(g.m_blocks);
+    g.M = rows;
+    g.split = 0;
+    g.layer = 0;
+    g.err = err;
+    launch_gemm_tc<EPI_STORE>(L, "img_in", ma, mb, mb, mh, g);
+}
+
+// v[r][:] = (LN(h[r]) (1 + scale_final)) W_out^T for rows [0, rows) of h.
+static void launch_final_tc(Launcher &L, const qi21_config &c, const float *h, int rows, const float *sf,
+                            const void *w_out, float *v, char *wsb, const WsLayout &lay, uint32_t *err) {
+    const int d = c.d_model;
+    bf16 *wp = (bf16 *)(wsb + lay.fwp);
+    float *u = (float *)(wsb + lay.fu), *part = (float *)(wsb + lay.fpart);
+    L.run("final_prep", [&] { k_final_prep<<<FT_C, 256, 0, L.st>>>((const bf16 *)w_out, sf, d, wp, u); });
+    CUtensorMap mh, mw;
+    if (!make_map2d(&mh, h, true, d, rows, 32, FT_BM) || !make_map2d(&mw, wp, false, d, FT_C, FT_BK, FT_C)) {
+        L.status = QI21_ERR_CUDA;
+        return;
+    }
+    const int mb = (rows + FT_BM - 1) / FT_BM, kblocks = d / FT_BK;
+    int ks = num_sms() / mb;
+    if (ks > FINAL_MAX_KSPLIT) ks = FINAL_MAX_KSPLIT;
+    if (ks > kblocks) ks = kblocks;
+    if (ks < 1) ks = 1;
+    FinalParams fp{rows, d, kblocks, ks, part, err};
+    static DeviceFlags attr;
+    smem_opt_in(k_final_tc, (int)FT_SMEM, attr);
+    L.run("final", [&] { k_final_tc<<<dim3(mb, ks), FT_THREADS, FT_SMEM, L.st>>>(mh, mw, fp); });
+    L.run("final_reduce", [&] {
+        k_final_reduce<<<(int)(((int64_t)rows * 16 + 255) / 256), 256, 0, L.st>>>(part, ks, rows, d, u, c.ln_eps, v);
+    });
 }
 
 template <typename T>
@@ -712,7 +828,11 @@ extern "C" qi21_status qi21_cached_step(const qi21_config *c, const qi21_weights
     }
     a.kv_limit = nullptr;
     a.kv_only_last = false;
-    if (c->dtype == QI21_DTYPE_BF16) {
+    if (c->dtype == QI21_DTYPE_BF16 && tc_head_supported(*c)) {
+        launch_img_in_tc(L, *c, x_k, w->w_img_in, a.h, B * N, (bf16 *)(wsb + lay.xin), a.err);
+        run_stack<bf16>(L, *c, *w, a);
+        launch_final_tc(L, *c, a.h, B * N, scale_final, w->w_out, v_out, wsb, lay, a.err);
+    } else if (c->dtype == QI21_DTYPE_BF16) {
         launch_img_in<bf16>(L, *c, x_k, w->w_img_in, a.h, B, N, N, 0);
         run_stack<bf16>(L, *c, *w, a);
         launch_final<bf16>(L, *c, a.h, N, 0, B, N, scale_final, w->w_out, v_out);

@@ -14,25 +14,32 @@
 //   EPI_RESIDUAL h[r][n] += tanh(gate)[n] * D[r][n]   (fp32 residual stream)
 //   EPI_SWIGLU   hid[r][j] = silu(D[r][j]) * D[r][F + j]   (gate and up halves
 //                of one 256-column tile come from W_gate and W_up rows j0..j0+127)
+//   EPI_STORE    out[r][n] = D[r][n] as fp32 through a TMA tensor store (img_in:
+//                the residual stream's first value, h = x W_img_in^T)
 #pragma once
 #include "qi21_sm100.cuh"
 
 namespace qi21 {
 
-enum { EPI_QKV = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2 };
+enum { EPI_QKV = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_STORE = 3 };
 
 constexpr int TC_BM = 128, TC_BN = 256, TC_BK = 64, TC_STAGES = 4;
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;          // 16 KB
 constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;          // 32 KB
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_THREADS = 192;
-// EPI_RESIDUAL stages each epilogue warp's 32 x 32 fp32 box in shared memory
-// (two buffers per warp) for the TMA reduce-add into the residual stream.
+// EPI_RESIDUAL and EPI_STORE stage each epilogue warp's 32 x 32 fp32 box in
+// shared memory (two buffers per warp) for the TMA reduce-add into the
+// residual stream, or the TMA store.
 constexpr int TC_RED_BUF = 32 * 32 * 4;
 constexpr int TC_RED_BYTES = 4 * 2 * TC_RED_BUF;
 template <int EPI>
+__host__ __device__ constexpr bool tc_boxed_epilogue() {
+    return EPI == EPI_RESIDUAL || EPI == EPI_STORE;
+}
+template <int EPI>
 constexpr size_t tc_smem_bytes() {
-    return 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + (EPI == EPI_RESIDUAL ? TC_RED_BYTES : 0) + 256;
+    return 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0) + 256;
 }
 
 struct GemmParams {
@@ -41,6 +48,7 @@ struct GemmParams {
     int m_blocks;      // ceil(R / 128)
     int n_blocks;      // output tiles along N
     int ksplit;        // EPI_RESIDUAL: K slices per output tile, each reduce-added into h (1 otherwise)
+    int sk_tiles;      // EPI_RESIDUAL with ksplit 1: the last sk_tiles tiles are shared stream-K style
     int group_m;       // row blocks per band of the tile order (0: all of them)
     int M, split;      // rows per item; rows m < split read the prefix modulation row
     // EPI_RESIDUAL
@@ -70,6 +78,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // out[box] += smem box, element-wise in L2 (2-D fp32 tensor map, 128B swizzle).
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *m, uint32_t src, int x, int y) {
     asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+// out[box] = smem box (2-D fp32 tensor map, 128B swizzle); rows past the
+// tensor's extent are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                      reinterpret_cast<uint64_t>(m)),
                  "r"(src), "r"(x), "r"(y)
                  : "memory");
@@ -118,6 +134,45 @@ __device__ __forceinline__ void tile_coords(const GemmParams &p, int tile, int k
     kb1 = (int)((int64_t)kblocks * (ks + 1) / p.ksplit);
 }
 
+// The work of one CTA: first the data-parallel units blockIdx.x, +gridDim.x, ...
+// (whole tiles, or K slices of them when ksplit > 1); then, when sk_tiles > 0
+// (residual epilogue, ksplit 1), this CTA's equal contiguous share of the K
+// blocks of the last sk_tiles tiles (stream-K: a share may start or end inside
+// a tile; every piece is reduce-added into h like a K slice). The data-parallel
+// units fill whole waves, so every CTA ends with the same number of K blocks.
+struct WorkCursor {
+    int unit;          // next data-parallel unit
+    int64_t it, end;   // stream-K iterations [it, end) of this CTA
+};
+
+__device__ __forceinline__ void work_begin(const GemmParams &p, int kblocks, WorkCursor &c) {
+    c.unit = blockIdx.x;
+    const int64_t W = (int64_t)p.sk_tiles * kblocks;
+    c.it = W * blockIdx.x / gridDim.x;
+    c.end = W * (blockIdx.x + 1) / gridDim.x;
+}
+
+__device__ __forceinline__ bool work_next(const GemmParams &p, int kblocks, WorkCursor &c, int &m_blk, int &n_blk,
+                                          int &kb0, int &kb1) {
+    const int dp_units = p.m_blocks * p.n_blocks * p.ksplit - p.sk_tiles;
+    if (c.unit < dp_units) {
+        tile_coords(p, c.unit, kblocks, m_blk, n_blk, kb0, kb1);
+        c.unit += gridDim.x;
+        return true;
+    }
+    if (c.it >= c.end) return false;
+    const int tile = dp_units + (int)(c.it / kblocks);
+    const int k0 = (int)(c.it % kblocks);
+    const int64_t left = c.end - c.it;
+    const int k1 = (left < (int64_t)(kblocks - k0)) ? k0 + (int)left : kblocks;
+    int unused0, unused1;
+    tile_coords(p, tile, kblocks, m_blk, n_blk, unused0, unused1);
+    kb0 = k0;
+    kb1 = k1;
+    c.it += k1 - k0;
+    return true;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -127,13 +182,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *stage_base = smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)TC_STAGES * TC_STAGE_BYTES +
-                                                  (EPI == EPI_RESIDUAL ? TC_RED_BYTES : 0));
+                                                  (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0));
     uint64_t *full = bars, *empty = bars + TC_STAGES, *tfull = bars + 2 * TC_STAGES, *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = p.m_blocks * p.n_blocks * p.ksplit;
     const int kblocks = p.K / TC_BK;
 
     if (threadIdx.x == 0) {
@@ -152,7 +206,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB0);
         tma_prefetch_desc(&tmB1);
-        if (EPI == EPI_QKV) tma_prefetch_desc(&tmB2);
+        if (EPI != EPI_SWIGLU) tma_prefetch_desc(&tmB2);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -169,9 +223,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                int m_blk, n_blk, kb0, kb1;
-                tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
+            WorkCursor wc;
+            work_begin(p, kblocks, wc);
+            int m_blk, n_blk, kb0, kb1;
+            while (ok && work_next(p, kblocks, wc, m_blk, n_blk, kb0, kb1)) {
                 const CUtensorMap *b0 = &tmB0, *b1 = &tmB1;
                 int rb0, rb1;
                 if (EPI == EPI_SWIGLU) {
@@ -221,9 +276,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint32_t phase = 0;
         int it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-            int m_blk, n_blk, kb0, kb1;
-            tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
+        WorkCursor wc;
+        work_begin(p, kblocks, wc);
+        int m_blk, n_blk, kb0, kb1;
+        for (; ok && work_next(p, kblocks, wc, m_blk, n_blk, kb0, kb1); ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             if (!wait_warp(&tempty[acc], acc_phase ^ 1)) break;
@@ -257,9 +313,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int row_in_tile = quad * 32 + lane;
         int it = 0;
         int red_count = 0;   // EPI_RESIDUAL: reduce-add boxes issued by this warp
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-            int m_blk, n_blk, kb0, kb1;
-            tile_coords(p, tile, kblocks, m_blk, n_blk, kb0, kb1);
+        WorkCursor wc;
+        work_begin(p, kblocks, wc);
+        int m_blk, n_blk, kb0, kb1;
+        for (; work_next(p, kblocks, wc, m_blk, n_blk, kb0, kb1); ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             // warp-uniform: the tcgen05.ld below is warp-collective
@@ -272,11 +329,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const int m = live ? r % p.M : 0;
             const int b = live ? r / p.M : 0;
             float v[32];
-            if (EPI == EPI_RESIDUAL) {
-                // h[r][n] += tanh(gate)[n] * acc: each warp writes its 32 rows x 32 columns
-                // into a swizzled shared box and one lane reduce-adds the box into h.
+            if (tc_boxed_epilogue<EPI>()) {
+                // EPI_RESIDUAL: h[r][n] += tanh(gate)[n] * acc; EPI_STORE: out[r][n] = acc.
+                // Each warp writes its 32 rows x 32 columns into a swizzled shared box
+                // and one lane reduce-adds (or stores) the box.
                 const int n0 = n_blk * TC_BN;
-                const float *g = (m < p.split ? p.g_lo : p.g_hi) + n0;
+                const float *g = EPI == EPI_RESIDUAL ? (m < p.split ? p.g_lo : p.g_hi) + n0 : nullptr;
                 uint8_t *stg = stage_base + (size_t)TC_STAGES * TC_STAGE_BYTES + (size_t)(warp - 2) * 2 * TC_RED_BUF;
                 const int sw = lane & 7;
 #pragma unroll 1
@@ -287,7 +345,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         tc_fence_before();
                         mbar_arrive(smem_u32(&tempty[acc]));
                     }
-                    if (live) {
+                    if (EPI == EPI_RESIDUAL && live) {
                         const float4 *g4 = reinterpret_cast<const float4 *>(g + cc * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -311,7 +369,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_reduce_add_2d(&tmB2, smem_u32(buf), n0 + cc * 32, m_blk * TC_BM + quad * 32);
+                        if (EPI == EPI_RESIDUAL)
+                            tma_reduce_add_2d(&tmB2, smem_u32(buf), n0 + cc * 32, m_blk * TC_BM + quad * 32);
+                        else
+                            tma_store_2d(&tmB2, smem_u32(buf), n0 + cc * 32, m_blk * TC_BM + quad * 32);
                         bulk_commit_group();
                     }
                 }
@@ -386,7 +447,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
         }
-        if (EPI == EPI_RESIDUAL && lane == 0) bulk_wait_group0();
+        if (tc_boxed_epilogue<EPI>() && lane == 0) bulk_wait_group0();
     }
     tc_fence_before();
     __syncthreads();

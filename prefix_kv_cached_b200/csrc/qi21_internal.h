@@ -20,8 +20,13 @@ namespace qi21 {
 //   kvf     : T [2][B][S][d]  K/V of the full recomputation
 //   gemm    : fp32 [R][max(3d, 2F)]  outputs of the CUDA-core GEMMs (present when
 //             they run: F32 mode, or BF16 mode with the tensor cores switched off)
+//   xin     : bf16 [B*N][C]   the latent rounded for the tensor-core img_in
+//   fwp, fu : bf16 [C][d], fp32 [C]  W_out scaled by (1 + scale_final) and its row
+//             sums (tensor-core final AdaLN + proj_out)
+//   fpart   : fp32 [FINAL_MAX_KSPLIT][B*N][68]  its per-K-slice partial sums
+constexpr int FINAL_MAX_KSPLIT = 8;
 struct WsLayout {
-    size_t err, gates, modtmp, h, xn, q, o, hid, kvf, gemm, total;
+    size_t err, gates, modtmp, h, xn, q, o, hid, kvf, gemm, xin, fwp, fu, fpart, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -81,6 +86,11 @@ inline WsLayout ws_layout(const qi21_config &c, int64_t B, int64_t P, int64_t N)
     L.kvf = take(eb * 2 * B * S * d);
     const int64_t gw = (3 * d > 2 * F) ? 3 * d : 2 * F;
     L.gemm = take(uses_cuda_core_gemm(c) ? sizeof(float) * R * gw : 0);
+    const int64_t C = c.latent_ch;
+    L.xin = take(2 * B * N * C);
+    L.fwp = take(2 * C * d);
+    L.fu = take(sizeof(float) * C);
+    L.fpart = take(sizeof(float) * FINAL_MAX_KSPLIT * B * N * 68);
     L.total = off;
     return L;
 }
