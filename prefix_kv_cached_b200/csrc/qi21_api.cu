@@ -167,15 +167,60 @@ static int num_sms() {
     return n;
 }
 
+#ifndef QI21_GEMM_PAIRS
+#define QI21_GEMM_PAIRS 1
+#endif
+
+// Row blocks per band of the GEMM tile order (0: one band). Up to 4096 rows one
+// band keeps the whole activation in L2 and reads each weight tile once per wave;
+// beyond that, bands of 2048 rows keep each wave's A rows in L2 (same-GPU A/B at
+// 16384 rows: gate/up -15 %, down -11 %, QKV -7 %; at 4096 rows banding cost
+// gate/up 3 %).
+static int gemm_group_m(int rows, int tile_rows) { return rows > 4096 ? 2048 / tile_rows : 0; }
+
+// The persistent tcgen05 GEMM over p.R rows. Work units are 256 x 256 tiles of a
+// CTA pair (cluster of 2) when there are at least two 128-row blocks, else
+// 128 x 256 tiles of single CTAs; one worker (pair or CTA) per pair of SMs or
+// SM. stream_k (residual epilogue): the tiles of the last, partial wave are
+// shared stream-K style so that every worker gets the same number of K blocks
+// and only about one extra partial tile per worker is reduce-added into h.
 template <int EPI>
 static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, const CUtensorMap &b0,
-                           const CUtensorMap &b1, const CUtensorMap &b2, const GemmParams &p) {
-    constexpr size_t smem = tc_smem_bytes<EPI>();
-    static DeviceFlags attr;
-    smem_opt_in(k_gemm_tc<EPI>, (int)smem, attr);
-    const int units = p.m_blocks * p.n_blocks * p.ksplit;
-    const int grid = (units < num_sms() && p.sk_tiles == 0) ? units : num_sms();
-    L.run(name, [&] { k_gemm_tc<EPI><<<grid, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
+                           const CUtensorMap &b1, const CUtensorMap &b2, GemmParams p, bool stream_k = false) {
+    const bool pair = QI21_GEMM_PAIRS && p.R > TC_BM;
+    const int tile_rows = pair ? 2 * TC_BM : TC_BM;
+    p.m_blocks = (p.R + tile_rows - 1) / tile_rows;
+    p.group_m = gemm_group_m(p.R, tile_rows);
+    const int workers = pair ? num_sms() / 2 : num_sms();
+    const int tiles = p.m_blocks * p.n_blocks;
+    p.sk_tiles = (stream_k && p.ksplit == 1) ? tiles % workers : 0;
+    const int units = tiles * p.ksplit;
+    const int active = (units < workers && p.sk_tiles == 0) ? units : workers;
+    if (pair) {
+        constexpr size_t smem = tc_smem_bytes<EPI, true>();
+        static DeviceFlags attr;
+        smem_opt_in(k_gemm_tc<EPI, true>, (int)smem, attr);
+        L.run(name, [&] {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * active);
+            cfg.blockDim = dim3(TC_THREADS);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = L.st;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = 2;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            cudaLaunchKernelEx(&cfg, k_gemm_tc<EPI, true>, a, b0, b1, b2, p);
+        });
+    } else {
+        constexpr size_t smem = tc_smem_bytes<EPI, false>();
+        static DeviceFlags attr;
+        smem_opt_in(k_gemm_tc<EPI, false>, (int)smem, attr);
+        L.run(name, [&] { k_gemm_tc<EPI, false><<<active, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
+    }
 }
 
 // 2-D fp32 tensor map [rows][inner] with a 32 x 32 box and 128-byte swizzle:
@@ -233,21 +278,6 @@ static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap 
     L.run("attn", [&] { k_attn_tc<DH><<<grid, Cf::THREADS, Cf::SMEM, L.st>>>(q, k, v, p); });
 }
 
-// Row blocks per band of the GEMM tile order: up to 32 row blocks (4096 rows) one
-// band keeps the whole activation in L2 and reads each weight tile once per wave;
-// beyond that, bands of 16 keep each wave's A rows in L2 (same-GPU A/B at 16384
-// rows: gate/up -15 %, down -11 %, QKV -7 %; at 4096 rows banding cost gate/up 3 %).
-static int gemm_group_m(int m_blocks) { return m_blocks > 32 ? 16 : 0; }
-
-// Residual GEMMs (the reduce-add epilogue sums partial products in L2): whole
-// tiles for the full waves of the persistent grid, and the tiles of the last,
-// partial wave shared stream-K style, so that every CTA gets the same number of
-// K blocks and only about one extra partial tile per CTA is reduce-added.
-static int residual_sk_tiles(int tiles) {
-    const int g = num_sms();
-    return tiles % g;
-}
-
 struct TcMaps {
     CUtensorMap xn, o, hid, wq, wk, wv, wo, wg, wu, wd, q4, k4, v4, h32;
 };
@@ -299,25 +329,14 @@ static void launch_modln(Launcher &L, const qi21_config &c, const float *h, T *o
     const int d = c.d_model;
     if (d % 4 == 0 && d <= 4 * 256 * 8) {
         const int vpt = (d / 4 + 255) / 256;
-        // as many blocks as fit on the GPU at once (each loops over rows)
-        auto grid_of = [&](auto kernel) {
-            static std::atomic<int> occ[kMaxDevices];
-            int dev = 0;
-            cudaGetDevice(&dev);
-            int per_sm = (dev >= 0 && dev < kMaxDevices) ? occ[dev].load() : 0;
-            if (per_sm <= 0) {
-                if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess ||
-                    per_sm <= 0)
-                    per_sm = 1;
-                if (dev >= 0 && dev < kMaxDevices) occ[dev].store(per_sm);
-            }
-            const int64_t g = (int64_t)per_sm * num_sms();
-            return (int)(rows < g ? rows : g);
-        };
+        // one row per block: measured alone at 4096 x 4096 it moves 4.9 TB/s (a
+        // plain fp32 -> bf16 copy of the same bytes: 5.6 TB/s); 128-thread blocks
+        // are as fast, 512 or 1024 threads, a warp per row, a one-pass
+        // (shifted) variance and a row-looping grid with the next row prefetched
+        // were slower
         L.run("modln", [&] {
-#define QI21_LN(V)                                                                                                \
-    k_modln_vec<T, V><<<grid_of(k_modln_vec<T, V>), 256, 0, L.st>>>(h, out, d, rows, M, split, sc_lo, sc_hi, sh_lo, \
-                                                                   sh_hi, c.ln_eps)
+#define QI21_LN(V)                                                                                           \
+    k_modln_vec<T, V><<<rows, 256, 0, L.st>>>(h, out, d, M, split, sc_lo, sc_hi, sh_lo, sh_hi, c.ln_eps)
             if (vpt <= 1) QI21_LN(1);
             else if (vpt <= 2) QI21_LN(2);
             else if (vpt <= 4) QI21_LN(4);
@@ -378,9 +397,7 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             return;
         }
         gp.R = R;
-        gp.m_blocks = (R + TC_BM - 1) / TC_BM;
         gp.ksplit = 1;
-        gp.group_m = gemm_group_m(gp.m_blocks);
         gp.M = a.M;
         gp.split = a.split;
         gp.h = a.h;
@@ -471,10 +488,9 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             GemmParams g = gp;
             g.K = d;
             g.n_blocks = d / TC_BN;
-            g.sk_tiles = residual_sk_tiles(g.m_blocks * g.n_blocks);
             g.g_lo = tg1_lo;
             g.g_hi = tg1_hi;
-            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.h32, g);
+            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_o", maps.o, maps.wo, maps.wo, maps.h32, g, true);
         } else {
             launch_gemm_simt<T>(L, o, d, Wo, d, a.gemm, d, R, d, d);
             L.run("gated_residual", [&] {
@@ -491,10 +507,9 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
             GemmParams g2 = gp;
             g2.K = F;
             g2.n_blocks = d / TC_BN;
-            g2.sk_tiles = residual_sk_tiles(g2.m_blocks * g2.n_blocks);
             g2.g_lo = tg2_lo;
             g2.g_hi = tg2_hi;
-            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.h32, g2);
+            launch_gemm_tc<EPI_RESIDUAL>(L, "gemm_down", maps.hid, maps.wd, maps.wd, maps.h32, g2, true);
         } else {
             launch_gemm_simt<T>(L, xn, d, Wg, d, a.gemm, 2 * F, R, F, d);
             launch_gemm_simt<T>(L, xn, d, Wu, d, a.gemm + F, 2 * F, R, F, d);
@@ -540,10 +555,8 @@ static void launch_img_in_tc(Launcher &L, const qi21_config &c, const float *x, 
     GemmParams g{};
     g.R = rows;
     g.K = C;
-    g.m_blocks = (rows + TC_BM - 1) / TC_BM;
     g.n_blocks = d / TC_BN;
     g.ksplit = 1;
-    g.group_m = gemm_group_m(g.m_blocks);
     g.M = rows;
     g.split = 0;
     g.layer = 0;

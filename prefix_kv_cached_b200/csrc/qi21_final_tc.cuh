@@ -39,16 +39,32 @@ struct FinalParams {
     uint32_t *err;
 };
 
-// W'[c][k] = bf16((1 + s[k]) W_out[c][k]); u[c] = sum_k W'[c][k] (fp32 sum of the rounded values).
+// W'[c][k] = bf16((1 + s[k]) W_out[c][k]); u[c] = sum_k W'[c][k] (fp32 sum of the
+// rounded values). One block per output c; each thread takes 8 consecutive k
+// (16-byte loads and stores), d % 8 == 0.
 static __global__ void __launch_bounds__(256) k_final_prep(const bf16 *__restrict__ w_out, const float *__restrict__ sf,
                                                            int d, bf16 *__restrict__ wp, float *__restrict__ u) {
     __shared__ float red[32];
     const int c = blockIdx.x;
+    const uint4 *w8 = reinterpret_cast<const uint4 *>(w_out + (size_t)c * d);
+    uint4 *o8 = reinterpret_cast<uint4 *>(wp + (size_t)c * d);
+    const float4 *s4 = reinterpret_cast<const float4 *>(sf);
     float acc = 0.f;
-    for (int k = threadIdx.x; k < d; k += blockDim.x) {
-        const bf16 w = __float2bfloat16_rn((1.f + sf[k]) * __bfloat162float(w_out[(size_t)c * d + k]));
-        wp[(size_t)c * d + k] = w;
-        acc += __bfloat162float(w);
+    for (int k8 = threadIdx.x; k8 < d / 8; k8 += blockDim.x) {
+        const uint4 wv = w8[k8];
+        const float4 sa = s4[2 * k8], sb = s4[2 * k8 + 1];
+        const float sc[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+        const uint32_t win[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t wout[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&win[i]));
+            const __nv_bfloat162 r = __floats2bfloat162_rn((1.f + sc[2 * i]) * f.x, (1.f + sc[2 * i + 1]) * f.y);
+            const float2 g = __bfloat1622float2(r);
+            acc += g.x + g.y;
+            wout[i] = *reinterpret_cast<const uint32_t *>(&r);
+        }
+        o8[k8] = make_uint4(wout[0], wout[1], wout[2], wout[3]);
     }
     acc = block_sum(acc, red);
     if (threadIdx.x == 0) u[c] = acc;

@@ -23,10 +23,8 @@ namespace qi21 {
 
 enum { EPI_QKV = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_STORE = 3 };
 
-constexpr int TC_BM = 128, TC_BN = 256, TC_BK = 64, TC_STAGES = 4;
-constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;          // 16 KB
-constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;          // 32 KB
-constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
+constexpr int TC_BM = 128, TC_BN = 256, TC_BK = 64;
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;          // 16 KB: a CTA's 128 rows of A per K block
 constexpr int TC_THREADS = 192;
 // EPI_RESIDUAL and EPI_STORE stage each epilogue warp's 32 x 32 fp32 box in
 // shared memory (two buffers per warp) for the TMA reduce-add into the
@@ -37,9 +35,25 @@ template <int EPI>
 __host__ __device__ constexpr bool tc_boxed_epilogue() {
     return EPI == EPI_RESIDUAL || EPI == EPI_STORE;
 }
-template <int EPI>
+
+// Shared-memory pipeline of one CTA. PAIR = false: the CTA computes a 128 x 256
+// tile alone and loads all 256 W rows of a K block. PAIR = true: two CTAs (a
+// cluster) compute a 256 x 256 tile with cta_group::2 MMAs; each loads its own
+// 128 rows of A and 128 of the 256 W rows, so a stage is 32 KB instead of 48 KB
+// and the shared-memory and L2 traffic per MMA drop by a third.
+template <int EPI, bool PAIR>
+struct TcCfg {
+    static constexpr int B_ROWS = PAIR ? 128 : 256;                 // W rows a CTA loads per K block
+    static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
+    static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
+    static constexpr int STAGES = PAIR ? (tc_boxed_epilogue<EPI>() ? 5 : 6) : 4;
+    static constexpr int TILE_ROWS = PAIR ? 256 : 128;              // output rows of a work unit
+    static constexpr size_t SMEM =
+        1024 + (size_t)STAGES * STAGE_BYTES + (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0) + 256;
+};
+template <int EPI, bool PAIR>
 constexpr size_t tc_smem_bytes() {
-    return 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0) + 256;
+    return TcCfg<EPI, PAIR>::SMEM;
 }
 
 struct GemmParams {
@@ -145,19 +159,20 @@ struct WorkCursor {
     int64_t it, end;   // stream-K iterations [it, end) of this CTA
 };
 
-__device__ __forceinline__ void work_begin(const GemmParams &p, int kblocks, WorkCursor &c) {
-    c.unit = blockIdx.x;
+// `worker` / `workers`: this CTA (or CTA pair) and how many there are.
+__device__ __forceinline__ void work_begin(const GemmParams &p, int kblocks, int worker, int workers, WorkCursor &c) {
+    c.unit = worker;
     const int64_t W = (int64_t)p.sk_tiles * kblocks;
-    c.it = W * blockIdx.x / gridDim.x;
-    c.end = W * (blockIdx.x + 1) / gridDim.x;
+    c.it = W * worker / workers;
+    c.end = W * (worker + 1) / workers;
 }
 
-__device__ __forceinline__ bool work_next(const GemmParams &p, int kblocks, WorkCursor &c, int &m_blk, int &n_blk,
-                                          int &kb0, int &kb1) {
+__device__ __forceinline__ bool work_next(const GemmParams &p, int kblocks, int workers, WorkCursor &c, int &m_blk,
+                                          int &n_blk, int &kb0, int &kb1) {
     const int dp_units = p.m_blocks * p.n_blocks * p.ksplit - p.sk_tiles;
     if (c.unit < dp_units) {
         tile_coords(p, c.unit, kblocks, m_blk, n_blk, kb0, kb1);
-        c.unit += gridDim.x;
+        c.unit += workers;
         return true;
     }
     if (c.it >= c.end) return false;
@@ -173,31 +188,39 @@ __device__ __forceinline__ bool work_next(const GemmParams &p, int kblocks, Work
     return true;
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
               const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2, GemmParams p) {
     using namespace sm100;
+    using Cfg = TcCfg<EPI, PAIR>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *stage_base = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)TC_STAGES * TC_STAGE_BYTES +
-                                                  (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0));
-    uint64_t *full = bars, *empty = bars + TC_STAGES, *tfull = bars + 2 * TC_STAGES, *tempty = tfull + 2;
+    uint8_t *red_base = smem + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(red_base + (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0));
+    uint64_t *full = bars, *empty = bars + Cfg::STAGES, *tfull = bars + 2 * Cfg::STAGES, *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    static_assert((2 * Cfg::STAGES + 4) * 8 + 8 <= 256, "barrier region");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int kblocks = p.K / TC_BK;
+    // CTA pair: rank 0 (the leader) issues every MMA of the pair; each CTA owns
+    // rows [rank * 128, rank * 128 + 128) of the 256-row tile.
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const int worker = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int workers = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const bool mma_cta = rank == 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < TC_STAGES; ++s) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 128);
+            mbar_init(smem_u32(&tempty[a]), PAIR ? 8 : 4);     // one arrival per epilogue warp of the tile
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -209,11 +232,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (EPI != EPI_SWIGLU) tma_prefetch_desc(&tmB2);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), 512);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_slot), 512);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), 512);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // the peer's barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -224,36 +253,48 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             WorkCursor wc;
-            work_begin(p, kblocks, wc);
+            work_begin(p, kblocks, worker, workers, wc);
             int m_blk, n_blk, kb0, kb1;
-            while (ok && work_next(p, kblocks, wc, m_blk, n_blk, kb0, kb1)) {
+            while (ok && work_next(p, kblocks, workers, wc, m_blk, n_blk, kb0, kb1)) {
+                // this CTA's W rows of the tile: all 256 (single CTA) or half of them (pair)
                 const CUtensorMap *b0 = &tmB0, *b1 = &tmB1;
                 int rb0, rb1;
                 if (EPI == EPI_SWIGLU) {
+                    // columns 0..127 of the tile from W_gate, 128..255 from W_up, rows j0..j0+127
                     rb0 = rb1 = n_blk * 128;
+                    if (PAIR && rank == 1) b0 = &tmB1;
                 } else if (EPI == EPI_QKV) {
                     const int n0 = n_blk * TC_BN, part = n0 / p.d;
                     const CUtensorMap *bm = part == 0 ? &tmB0 : (part == 1 ? &tmB1 : &tmB2);
                     b0 = b1 = bm;
-                    rb0 = n0 - part * p.d;
+                    rb0 = n0 - part * p.d + (int)rank * 128;
                     rb1 = rb0 + 128;
                 } else {
-                    rb0 = n_blk * TC_BN;
+                    rb0 = n_blk * TC_BN + (int)rank * 128;
                     rb1 = rb0 + 128;
                 }
+                const int arow = m_blk * Cfg::TILE_ROWS + (int)rank * TC_BM;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = smem_u32(&full[stage]);
-                    mbar_arrive_expect_tx(fb, TC_STAGE_BYTES);
-                    const uint32_t sa = smem_u32(stage_base + (size_t)stage * TC_STAGE_BYTES);
+                    const uint32_t sa = smem_u32(stage_base + (size_t)stage * Cfg::STAGE_BYTES);
                     const uint32_t sb = sa + TC_A_BYTES;
-                    tma_load_3d(sa, &tmA, fb, kb * TC_BK, m_blk * TC_BM, 0);
-                    tma_load_3d(sb, b0, fb, kb * TC_BK, rb0, p.layer);
-                    tma_load_3d(sb + TC_B_BYTES / 2, b1, fb, kb * TC_BK, rb1, p.layer);
-                    if (++stage == TC_STAGES) {
+                    if constexpr (PAIR) {
+                        // both CTAs' loads complete on the leader's full barrier
+                        const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                        if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * Cfg::STAGE_BYTES);
+                        tma_load_3d_pair(sa, &tmA, fb, kb * TC_BK, arow, 0);
+                        tma_load_3d_pair(sb, b0, fb, kb * TC_BK, rb0, p.layer);
+                    } else {
+                        const uint32_t fb = smem_u32(&full[stage]);
+                        mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+                        tma_load_3d(sa, &tmA, fb, kb * TC_BK, arow, 0);
+                        tma_load_3d(sb, b0, fb, kb * TC_BK, rb0, p.layer);
+                        tma_load_3d(sb + Cfg::B_BYTES / 2, b1, fb, kb * TC_BK, rb1, p.layer);
+                    }
+                    if (++stage == Cfg::STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
@@ -261,70 +302,97 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------- UMMA issuer
+        // ---------------------------------------------------------- UMMA issuer (the leader CTA's)
         // The whole warp runs the schedule and one elected lane issues; the
         // operand descriptors are built once and advanced by adding to the
         // start-address field (16-byte units: 32 B per K=16 step).
-        constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN);
-        constexpr uint32_t STAGE_UNITS = TC_STAGE_BYTES >> 4, A_UNITS = TC_A_BYTES >> 4;
-        const uint64_t d0 = sdesc_kmajor_sw128(smem_u32(stage_base));
-        const bool leader = elect_one();
-        auto wait_warp = [&](uint64_t *bar, uint32_t parity) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag, p.err) ? 1 : 0) != 0;
-        };
-        int stage = 0;
-        uint32_t phase = 0;
-        int it = 0;
-        bool ok = true;
-        WorkCursor wc;
-        work_begin(p, kblocks, wc);
-        int m_blk, n_blk, kb0, kb1;
-        for (; ok && work_next(p, kblocks, wc, m_blk, n_blk, kb0, kb1); ++it) {
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
-            if (!wait_warp(&tempty[acc], acc_phase ^ 1)) break;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (!wait_warp(&full[stage], phase)) {
-                    ok = false;
-                    break;
-                }
+        if (mma_cta) {
+            constexpr uint32_t idesc = idesc_bf16_f32(Cfg::TILE_ROWS, TC_BN);
+            constexpr uint32_t STAGE_UNITS = Cfg::STAGE_BYTES >> 4, A_UNITS = TC_A_BYTES >> 4;
+            const uint64_t d0 = sdesc_kmajor_sw128(smem_u32(stage_base));
+            const bool leader = elect_one();
+            auto wait_warp = [&](uint64_t *bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort_flag, p.err) ? 1 : 0) != 0;
+            };
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            WorkCursor wc;
+            work_begin(p, kblocks, worker, workers, wc);
+            int m_blk, n_blk, kb0, kb1;
+            for (; ok && work_next(p, kblocks, workers, wc, m_blk, n_blk, kb0, kb1); ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!wait_warp(&tempty[acc], acc_phase ^ 1)) break;
                 tc_fence_after();
-                if (leader) {
-                    const uint64_t da = d0 + (uint32_t)stage * STAGE_UNITS;
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!wait_warp(&full[stage], phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (leader) {
+                        const uint64_t da = d0 + (uint32_t)stage * STAGE_UNITS;
 #pragma unroll
-                    for (int k = 0; k < TC_BK / 16; ++k)
-                        umma_f16(d_tmem, da + 2 * k, da + A_UNITS + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-                    umma_commit(smem_u32(&empty[stage]));
+                        for (int k = 0; k < TC_BK / 16; ++k) {
+                            if constexpr (PAIR)
+                                umma_f16_pair(d_tmem, da + 2 * k, da + A_UNITS + 2 * k, idesc,
+                                              (kb > kb0 || k > 0) ? 1u : 0u);
+                            else
+                                umma_f16(d_tmem, da + 2 * k, da + A_UNITS + 2 * k, idesc,
+                                         (kb > kb0 || k > 0) ? 1u : 0u);
+                        }
+                        if constexpr (PAIR)
+                            umma_commit_pair(smem_u32(&empty[stage]), 0x3);
+                        else
+                            umma_commit(smem_u32(&empty[stage]));
+                    }
+                    __syncwarp();
+                    if (++stage == Cfg::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (ok && leader) {
+                    if constexpr (PAIR)
+                        umma_commit_pair(smem_u32(&tfull[acc]), 0x3);
+                    else
+                        umma_commit(smem_u32(&tfull[acc]));
                 }
                 __syncwarp();
-                if (++stage == TC_STAGES) {
-                    stage = 0;
-                    phase ^= 1;
-                }
             }
-            if (ok && leader) umma_commit(smem_u32(&tfull[acc]));
-            __syncwarp();
         }
     } else {
         // ---------------------------------------------------------- epilogue (warps 2..5)
         const int quad = warp & 3;
-        const int row_in_tile = quad * 32 + lane;
+        const int row_in_tile = (int)rank * TC_BM + quad * 32 + lane;
         int it = 0;
-        int red_count = 0;   // EPI_RESIDUAL: reduce-add boxes issued by this warp
+        int red_count = 0;   // boxed epilogues: reduce-add / store boxes issued by this warp
         WorkCursor wc;
-        work_begin(p, kblocks, wc);
+        work_begin(p, kblocks, worker, workers, wc);
         int m_blk, n_blk, kb0, kb1;
-        for (; work_next(p, kblocks, wc, m_blk, n_blk, kb0, kb1); ++it) {
+        for (; work_next(p, kblocks, workers, wc, m_blk, n_blk, kb0, kb1); ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             // warp-uniform: the tcgen05.ld below is warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.err) ? 1 : 0))
                 break;
             tc_fence_after();
+            // this warp is done with the accumulator: tell the leader's MMA warp
+            auto release_acc = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR)
+                        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+                    else
+                        mbar_arrive(smem_u32(&tempty[acc]));
+                }
+            };
             const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * TC_BN);
-            const int r = m_blk * TC_BM + row_in_tile;
+            const int r = m_blk * Cfg::TILE_ROWS + row_in_tile;
             const bool live = r < p.R;
             const int m = live ? r % p.M : 0;
             const int b = live ? r / p.M : 0;
@@ -335,16 +403,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 // and one lane reduce-adds (or stores) the box.
                 const int n0 = n_blk * TC_BN;
                 const float *g = EPI == EPI_RESIDUAL ? (m < p.split ? p.g_lo : p.g_hi) + n0 : nullptr;
-                uint8_t *stg = stage_base + (size_t)TC_STAGES * TC_STAGE_BYTES + (size_t)(warp - 2) * 2 * TC_RED_BUF;
+                uint8_t *stg = red_base + (size_t)(warp - 2) * 2 * TC_RED_BUF;
                 const int sw = lane & 7;
+                const int box_row = m_blk * Cfg::TILE_ROWS + (int)rank * TC_BM + quad * 32;
 #pragma unroll 1
                 for (int cc = 0; cc < TC_BN / 32; ++cc, ++red_count) {
                     tmem_ld32(t_row + cc * 32, v);
                     tmem_wait_ld();
-                    if (cc == TC_BN / 32 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(smem_u32(&tempty[acc]));
-                    }
+                    if (cc == TC_BN / 32 - 1) release_acc();
                     if (EPI == EPI_RESIDUAL && live) {
                         const float4 *g4 = reinterpret_cast<const float4 *>(g + cc * 32);
 #pragma unroll
@@ -370,13 +436,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     __syncwarp();
                     if (lane == 0) {
                         if (EPI == EPI_RESIDUAL)
-                            tma_reduce_add_2d(&tmB2, smem_u32(buf), n0 + cc * 32, m_blk * TC_BM + quad * 32);
+                            tma_reduce_add_2d(&tmB2, smem_u32(buf), n0 + cc * 32, box_row);
                         else
-                            tma_store_2d(&tmB2, smem_u32(buf), n0 + cc * 32, m_blk * TC_BM + quad * 32);
+                            tma_store_2d(&tmB2, smem_u32(buf), n0 + cc * 32, box_row);
                         bulk_commit_group();
                     }
                 }
-                continue;   // TMEM already released
+                continue;   // accumulator already released
             } else if (EPI == EPI_SWIGLU) {
                 const int j0 = n_blk * 128;
                 float u[32];
@@ -444,16 +510,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&tempty[acc]));
+            release_acc();
         }
         if (tc_boxed_epilogue<EPI>() && lane == 0) bulk_wait_group0();
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // neither CTA frees the pair's TMEM while the other still uses it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        if constexpr (PAIR)
+            tmem_dealloc_pair(tmem_base, 512);
+        else
+            tmem_dealloc(tmem_base, 512);
     }
 }
 

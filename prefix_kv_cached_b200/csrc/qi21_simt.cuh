@@ -25,83 +25,65 @@ static __global__ void k_prep_gates(const float *__restrict__ mod_lo, const floa
 }
 
 // ---------------------------------------------------------------------------
-// Modulated LayerNorm: out = LN(h) * (1 + scale) (+ shift).
+// Modulated LayerNorm: out = LN(h) * (1 + scale) (+ shift), one row per block.
 // Row r is token m = r % M of its item; m < split reads the prefix row (lo),
 // otherwise the target row (hi) — the per-token row selection of the 3B page.
-// Two-pass mean/variance in fp32 over a register copy of the row (VPT float4
-// per thread, 256 threads). A block handles rows blockIdx.x, +gridDim.x, ...
-// (the grid is sized to the blocks that fit on the GPU at once) and issues
-// the loads of its next row before reducing the current one, so that HBM
-// reads stay in flight through the two block reductions and the stores.
+// Two-pass mean/variance in fp32 over a register copy of the row.
 // ---------------------------------------------------------------------------
-template <int VPT>
-__device__ __forceinline__ void modln_load_row(const float *__restrict__ h, size_t row, int n4, float4 (&v)[VPT]) {
-    const float4 *x4 = reinterpret_cast<const float4 *>(h + row * (size_t)(n4 * 4));
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int c4 = threadIdx.x + i * 256;
-        v[i] = c4 < n4 ? x4[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-}
-
 template <typename T, int VPT>
-__global__ void __launch_bounds__(256) k_modln_vec(const float *__restrict__ h, T *__restrict__ out, int d, int rows,
-                                                   int M, int split, const float *__restrict__ scale_lo,
+__global__ void __launch_bounds__(256) k_modln_vec(const float *__restrict__ h, T *__restrict__ out, int d, int M,
+                                                   int split, const float *__restrict__ scale_lo,
                                                    const float *__restrict__ scale_hi,
                                                    const float *__restrict__ shift_lo,
                                                    const float *__restrict__ shift_hi, float eps) {
     __shared__ float red[32];
+    const int r = blockIdx.x;
+    const int m = r % M;
+    const float *sc = m < split ? scale_lo : scale_hi;
+    const float *sh = m < split ? shift_lo : shift_hi;
+    const float4 *x4 = reinterpret_cast<const float4 *>(h + (size_t)r * d);
     const int n4 = d >> 2;
-    float4 v[VPT], nxt[VPT];
-    int r = blockIdx.x;
-    if (r < rows) modln_load_row<VPT>(h, (size_t)r, n4, v);
-    for (; r < rows; r += gridDim.x) {
-        const int rn = r + gridDim.x;
-        if (rn < rows) modln_load_row<VPT>(h, (size_t)rn, n4, nxt);
-        const int m = r % M;
-        const float *sc = m < split ? scale_lo : scale_hi;
-        const float *sh = m < split ? shift_lo : shift_hi;
-        float s = 0.f;
+    float4 v[VPT];
+    float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-        const float mean = block_sum(s, red) / d;
-        float q = 0.f;
+    for (int i = 0; i < VPT; ++i) {
+        const int c4 = threadIdx.x + i * 256;
+        v[i] = c4 < n4 ? x4[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    }
+    const float mean = block_sum(s, red) / d;
+    float q = 0.f;
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int c4 = threadIdx.x + i * 256;
-            if (c4 < n4) {
-                const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, e = v[i].w - mean;
-                q += (a * a + b * b) + (c * c + e * e);
-            }
+    for (int i = 0; i < VPT; ++i) {
+        const int c4 = threadIdx.x + i * 256;
+        if (c4 < n4) {
+            const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, e = v[i].w - mean;
+            q += (a * a + b * b) + (c * c + e * e);
         }
-        const float var = block_sum(q, red) / d;
-        const float rstd = 1.0f / sqrtf(var + eps);
+    }
+    const float var = block_sum(q, red) / d;
+    const float rstd = 1.0f / sqrtf(var + eps);
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int c4 = threadIdx.x + i * 256;
-            if (c4 < n4) {
-                const float4 s4 = reinterpret_cast<const float4 *>(sc)[c4];
-                float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (sh) b4 = reinterpret_cast<const float4 *>(sh)[c4];
-                float y0 = (v[i].x - mean) * rstd * (1.f + s4.x) + b4.x;
-                float y1 = (v[i].y - mean) * rstd * (1.f + s4.y) + b4.y;
-                float y2 = (v[i].z - mean) * rstd * (1.f + s4.z) + b4.z;
-                float y3 = (v[i].w - mean) * rstd * (1.f + s4.w) + b4.w;
-                T *o = out + (size_t)r * d + 4 * c4;
-                if constexpr (sizeof(T) == 2) {
-                    __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1), p1 = __floats2bfloat162_rn(y2, y3);
-                    uint2 pk;
-                    pk.x = *reinterpret_cast<uint32_t *>(&p0);
-                    pk.y = *reinterpret_cast<uint32_t *>(&p1);
-                    *reinterpret_cast<uint2 *>(o) = pk;
-                } else {
-                    *reinterpret_cast<float4 *>(o) = make_float4(y0, y1, y2, y3);
-                }
+    for (int i = 0; i < VPT; ++i) {
+        const int c4 = threadIdx.x + i * 256;
+        if (c4 < n4) {
+            const float4 s4 = reinterpret_cast<const float4 *>(sc)[c4];
+            float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (sh) b4 = reinterpret_cast<const float4 *>(sh)[c4];
+            float y0 = (v[i].x - mean) * rstd * (1.f + s4.x) + b4.x;
+            float y1 = (v[i].y - mean) * rstd * (1.f + s4.y) + b4.y;
+            float y2 = (v[i].z - mean) * rstd * (1.f + s4.z) + b4.z;
+            float y3 = (v[i].w - mean) * rstd * (1.f + s4.w) + b4.w;
+            T *o = out + (size_t)r * d + 4 * c4;
+            if constexpr (sizeof(T) == 2) {
+                __nv_bfloat162 p0 = __floats2bfloat162_rn(y0, y1), p1 = __floats2bfloat162_rn(y2, y3);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t *>(&p0);
+                pk.y = *reinterpret_cast<uint32_t *>(&p1);
+                *reinterpret_cast<uint2 *>(o) = pk;
+            } else {
+                *reinterpret_cast<float4 *>(o) = make_float4(y0, y1, y2, y3);
             }
-        }
-        if (rn < rows) {
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) v[i] = nxt[i];
         }
     }
 }

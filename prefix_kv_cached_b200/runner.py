@@ -48,6 +48,8 @@ class Qi21Runner:
         self.dtype = dtype
         self.tdtype = _TORCH_DTYPE[dtype]
         self.device = torch.device(device)
+        if self.device.type == "cuda" and self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         self.cfg = make_config(self.shape, dtype)
         sh = self.shape
         self.meta = B.qi21_build_metadata(list(workload.segments), frame_mode)

@@ -269,3 +269,23 @@ def test_noalloc_applies_the_modulation_shape_checks(B):
     bad = make_config(C.SMALL, B.QI21_DTYPE_F32)
     bad.n_heads = 3
     assert B.qi21_modulation_noalloc(bad, w, 500.0, fake, fake, 0) == B.QI21_ERR_SHAPE
+
+
+def test_runner_checks_caller_weights_on_its_device(B):
+    """The runner takes the caller's weights as they are (no drawing, no
+    conversion): tensors of the storage dtype on its device; anything else is
+    refused. Host-only: a runner on the CPU device builds its metadata, RoPE
+    table and cache descriptor without touching a GPU."""
+    import torch
+    from prefix_kv_cached_b200.runner import Qi21Runner
+    w = C.make_workload("toy")
+    wts = C.host_weights(w, "float32")
+    r = Qi21Runner(w, B.QI21_DTYPE_F32, device="cpu", host_weights=wts)
+    assert (r.P, r.N) == (7, 4) and r.weights["w_q"].dtype == torch.float32
+    tw = {k: torch.from_numpy(v).float() for k, v in wts.items()}
+    Qi21Runner(w, B.QI21_DTYPE_F32, device="cpu", weights=tw)
+    bad = dict(tw, w_q=tw["w_q"].double())
+    with pytest.raises(ValueError):
+        Qi21Runner(w, B.QI21_DTYPE_F32, device="cpu", weights=bad)
+    with pytest.raises(ValueError):
+        Qi21Runner(w, B.QI21_DTYPE_F32, device="cpu", weights=tw, host_weights=wts)
