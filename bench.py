@@ -613,10 +613,26 @@ def main():
     B.qi21_profile_enable(0)
     prof = B.qi21_profile_read()
     ms = t0.elapsed_time(t1)
+    launches_timed = launches[0]
     tokens = w.batch * w.n_target
     ms_max, value = aggregate(world, tokens, args.steps, ms)
     r.check_device()
     ms_step = ms_max / args.steps
+
+    # the same steps again without the per-launch CUDA events (which sit between
+    # the kernels in the stream): what the instrumentation itself costs
+    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    u0.record(st)
+    for k in range(args.steps):
+        step(k)
+    u1.record(st)
+    torch.cuda.synchronize()
+    r.check_device()
+    ums_max, uvalue = aggregate(world, tokens, args.steps, u0.elapsed_time(u1))
+    uninstrumented = {"ms_per_step": round(ums_max / args.steps, 3), "value": round(uvalue, 1),
+                      "how": "the timed steps repeated right after, without the per-launch timing events"}
     per_step = [t0.elapsed_time(marks[0])] + [marks[i - 1].elapsed_time(marks[i]) for i in range(1, len(marks))]
     pct = {f"p{q}": round(float(np.percentile(per_step, q)), 3) for q in (50, 95, 99)}
 
@@ -752,11 +768,12 @@ def main():
             "tensor_frac_step_per_clock": step_fr.get("frac_per_clock_vs_sustained"),
             "step_tflops": round(step_tflops, 1),
             "step_ms_percentiles": pct,
+            "uninstrumented": uninstrumented,
             "batched_shared_prefix": batched,
             "per_image": {"extract_ms": round(extract_ms, 3),
                           "tokens_per_s": round(world * tokens / ((extract_ms + 8 * ms_step) / 1e3), 1),
                           "graph": image},
-            "roofline": roof, "kernels": kernels, "gpu_launches": launches[0], "clocks": clk, "e2e": e2e,
+            "roofline": roof, "kernels": kernels, "gpu_launches": launches_timed, "clocks": clk, "e2e": e2e,
             "configs": other_configs,
         }
         if world == 1 and not args.no_cpu_baseline:

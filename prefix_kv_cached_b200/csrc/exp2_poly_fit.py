@@ -1,5 +1,6 @@
 """Coefficients of the degree-3 polynomial the attention softmax uses for part
-of its exp2 evaluations (the rest run on the MUFU unit).
+of its exp2 evaluations (ex2_poly2 in qi21_attn_tc.cuh, every 8th pair of a
+row; the rest run on the MUFU unit).
 
 Method: Cody-Waite style argument split 2^x = 2^n * 2^f with n = rint(x),
 f = x - n in [-1/2, 1/2]; 2^f is approximated by the cubic that minimises the

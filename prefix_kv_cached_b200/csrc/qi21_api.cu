@@ -95,6 +95,35 @@ struct Launcher {
 
 static inline bool al16(const void *p) { return p && ((uintptr_t)p & 15) == 0; }
 
+#ifndef QI21_PDL
+#define QI21_PDL 0
+#endif
+
+// Launch a kernel that calls pdl_wait() before its first global-memory access
+// with programmatic stream serialisation, so that it may be scheduled (and run
+// its prologue) while the previous kernel in the stream finishes. Optional
+// extra attribute (the GEMM's cluster shape).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dep(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              const cudaLaunchAttribute *extra, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    int n = 0;
+    if (QI21_PDL) {
+        at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (extra) at[n++] = *extra;
+    cfg.attrs = at;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // The dynamic shared-memory opt-in above 48 KB is a per-device attribute of a
 // kernel: each call site keeps one flag per device and sets it on the current
 // device the first time (the call is not a stream operation, so this also
@@ -179,15 +208,18 @@ static int num_sms() {
 static int gemm_group_m(int rows, int tile_rows) { return rows > 4096 ? 2048 / tile_rows : 0; }
 
 // The persistent tcgen05 GEMM over p.R rows. Work units are 256 x 256 tiles of a
-// CTA pair (cluster of 2) when there are at least two 128-row blocks, else
-// 128 x 256 tiles of single CTAs; one worker (pair or CTA) per pair of SMs or
-// SM. stream_k (residual epilogue): the tiles of the last, partial wave are
-// shared stream-K style so that every worker gets the same number of K blocks
-// and only about one extra partial tile per worker is reduce-added into h.
+// CTA pair (cluster of 2) from 4096 rows on, else 128 x 256 tiles of single CTAs;
+// one worker (pair or CTA) per pair of SMs or SM. Same-GPU A/B at 4096 rows
+// (d 4096): pairs took QKV 300 -> 252 us, gate/up 554 -> 497, down 311 -> 275,
+// out-proj 111 -> 97; at 2048 rows (d 1024) they were 3-11 % slower (half as
+// many work units), and for img_in (K = 64) 27 vs 21 us. stream_k (residual
+// epilogue): the tiles of the last, partial wave are shared stream-K style so
+// that every worker gets the same number of K blocks and only about one extra
+// partial tile per worker is reduce-added into h.
 template <int EPI>
 static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, const CUtensorMap &b0,
                            const CUtensorMap &b1, const CUtensorMap &b2, GemmParams p, bool stream_k = false) {
-    const bool pair = QI21_GEMM_PAIRS && p.R > TC_BM;
+    const bool pair = QI21_GEMM_PAIRS && EPI != EPI_STORE && p.R >= 4096;
     const int tile_rows = pair ? 2 * TC_BM : TC_BM;
     p.m_blocks = (p.R + tile_rows - 1) / tile_rows;
     p.group_m = gemm_group_m(p.R, tile_rows);
@@ -200,26 +232,17 @@ static void launch_gemm_tc(Launcher &L, const char *name, const CUtensorMap &a, 
         constexpr size_t smem = tc_smem_bytes<EPI, true>();
         static DeviceFlags attr;
         smem_opt_in(k_gemm_tc<EPI, true>, (int)smem, attr);
-        L.run(name, [&] {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(2 * active);
-            cfg.blockDim = dim3(TC_THREADS);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = L.st;
-            cudaLaunchAttribute at[1];
-            at[0].id = cudaLaunchAttributeClusterDimension;
-            at[0].val.clusterDim.x = 2;
-            at[0].val.clusterDim.y = 1;
-            at[0].val.clusterDim.z = 1;
-            cfg.attrs = at;
-            cfg.numAttrs = 1;
-            cudaLaunchKernelEx(&cfg, k_gemm_tc<EPI, true>, a, b0, b1, b2, p);
-        });
+        cudaLaunchAttribute cl;
+        cl.id = cudaLaunchAttributeClusterDimension;
+        cl.val.clusterDim.x = 2;
+        cl.val.clusterDim.y = 1;
+        cl.val.clusterDim.z = 1;
+        L.run(name, [&] { launch_dep(k_gemm_tc<EPI, true>, dim3(2 * active), dim3(TC_THREADS), smem, L.st, &cl, a, b0, b1, b2, p); });
     } else {
         constexpr size_t smem = tc_smem_bytes<EPI, false>();
         static DeviceFlags attr;
         smem_opt_in(k_gemm_tc<EPI, false>, (int)smem, attr);
-        L.run(name, [&] { k_gemm_tc<EPI, false><<<active, TC_THREADS, smem, L.st>>>(a, b0, b1, b2, p); });
+        L.run(name, [&] { launch_dep(k_gemm_tc<EPI, false>, dim3(active), dim3(TC_THREADS), smem, L.st, nullptr, a, b0, b1, b2, p); });
     }
 }
 
@@ -275,7 +298,7 @@ static void launch_attn_tc(Launcher &L, const CUtensorMap &q, const CUtensorMap 
     static DeviceFlags attr;
     smem_opt_in(k_attn_tc<DH>, (int)Cf::SMEM, attr);
     dim3 grid((p.Mq + Cf::BQ - 1) / Cf::BQ, p.H, B);
-    L.run("attn", [&] { k_attn_tc<DH><<<grid, Cf::THREADS, Cf::SMEM, L.st>>>(q, k, v, p); });
+    L.run("attn", [&] { launch_dep(k_attn_tc<DH>, grid, dim3(Cf::THREADS), Cf::SMEM, L.st, nullptr, q, k, v, p); });
 }
 
 struct TcMaps {
@@ -336,7 +359,8 @@ static void launch_modln(Launcher &L, const qi21_config &c, const float *h, T *o
         // were slower
         L.run("modln", [&] {
 #define QI21_LN(V)                                                                                           \
-    k_modln_vec<T, V><<<rows, 256, 0, L.st>>>(h, out, d, M, split, sc_lo, sc_hi, sh_lo, sh_hi, c.ln_eps)
+    launch_dep(k_modln_vec<T, V>, dim3(rows), dim3(256), 0, L.st, nullptr, h, out, d, M, split, sc_lo, sc_hi, sh_lo, \
+               sh_hi, c.ln_eps)
             if (vpt <= 1) QI21_LN(1);
             else if (vpt <= 2) QI21_LN(2);
             else if (vpt <= 4) QI21_LN(4);
@@ -415,7 +439,8 @@ static void run_stack(Launcher &L, const qi21_config &c, const qi21_weights &w, 
     }
 
     L.run("prep_gates", [&] {
-        k_prep_gates<<<grid_for(d, 256), 256, 0, L.st>>>(a.mod_lo, a.mod_hi, d, c.use_shift, a.gates);
+        launch_dep(k_prep_gates, dim3(grid_for(d, 256)), dim3(256), 0, L.st, nullptr, a.mod_lo, a.mod_hi, d, c.use_shift,
+                   a.gates);
     });
     for (int l = 0; l < c.n_layers; ++l) {
         const T *Wq = (const T *)w.w_q + (size_t)l * d * d, *Wk = (const T *)w.w_k + (size_t)l * d * d;
@@ -533,6 +558,8 @@ static bool tc_head_supported(const qi21_config &c) {
 }
 
 static __global__ void k_to_bf16(const float *__restrict__ x, bf16 *__restrict__ y, int64_t n4) {
+    pdl_launch_dependents();
+    pdl_wait();
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
         const float4 f = reinterpret_cast<const float4 *>(x)[i];
         reinterpret_cast<uint2 *>(y)[i] = make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
@@ -545,7 +572,7 @@ static void launch_img_in_tc(Launcher &L, const qi21_config &c, const float *x, 
                              int rows, bf16 *xin, uint32_t *err) {
     const int d = c.d_model, C = c.latent_ch;
     const int64_t n4 = (int64_t)rows * C / 4;
-    L.run("img_in_cvt", [&] { k_to_bf16<<<grid_for(n4, 256), 256, 0, L.st>>>(x, xin, n4); });
+    L.run("img_in_cvt", [&] { launch_dep(k_to_bf16, dim3(grid_for(n4, 256)), dim3(256), 0, L.st, nullptr, x, xin, n4); });
     CUtensorMap ma, mb, mh;
     if (!make_map(&ma, xin, C, rows, 1, 128) || !make_map(&mb, w_img_in, C, d, 1, 128) ||
         !make_map_f32(&mh, h, d, rows)) {
@@ -570,7 +597,9 @@ static void launch_final_tc(Launcher &L, const qi21_config &c, const float *h, i
     const int d = c.d_model;
     bf16 *wp = (bf16 *)(wsb + lay.fwp);
     float *u = (float *)(wsb + lay.fu), *part = (float *)(wsb + lay.fpart);
-    L.run("final_prep", [&] { k_final_prep<<<FT_C, 256, 0, L.st>>>((const bf16 *)w_out, sf, d, wp, u); });
+    L.run("final_prep", [&] {
+        launch_dep(k_final_prep, dim3(FT_C), dim3(256), 0, L.st, nullptr, (const bf16 *)w_out, sf, d, wp, u);
+    });
     CUtensorMap mh, mw;
     if (!make_map2d(&mh, h, true, d, rows, 32, FT_BM) || !make_map2d(&mw, wp, false, d, FT_C, FT_BK, FT_C)) {
         L.status = QI21_ERR_CUDA;
@@ -584,9 +613,10 @@ static void launch_final_tc(Launcher &L, const qi21_config &c, const float *h, i
     FinalParams fp{rows, d, kblocks, ks, part, err};
     static DeviceFlags attr;
     smem_opt_in(k_final_tc, (int)FT_SMEM, attr);
-    L.run("final", [&] { k_final_tc<<<dim3(mb, ks), FT_THREADS, FT_SMEM, L.st>>>(mh, mw, fp); });
+    L.run("final", [&] { launch_dep(k_final_tc, dim3(mb, ks), dim3(FT_THREADS), FT_SMEM, L.st, nullptr, mh, mw, fp); });
     L.run("final_reduce", [&] {
-        k_final_reduce<<<(int)(((int64_t)rows * 16 + 255) / 256), 256, 0, L.st>>>(part, ks, rows, d, u, c.ln_eps, v);
+        launch_dep(k_final_reduce, dim3((int)(((int64_t)rows * 16 + 255) / 256)), dim3(256), 0, L.st, nullptr, part,
+                   ks, rows, d, u, c.ln_eps, v);
     });
 }
 
@@ -686,18 +716,22 @@ static qi21_status modulation_impl(const qi21_config *c, const qi21_weights *w, 
         static DeviceFlags attr;
         smem_opt_in(k_gemv2<T>, 64 * 1024, attr);
         if (emb)
-            L.run("temb_in", [&] { k_temb_in<T><<<(d + 7) / 8, 256, 0, st>>>((const T *)w->w_t1, *emb, K0, d, a1); });
+            L.run("temb_in", [&] {
+                launch_dep(k_temb_in<T>, dim3((d + 7) / 8), dim3(256), 0, st, nullptr, (const T *)w->w_t1, *emb, K0, d,
+                           a1);
+            });
         else
             L.run("temb_in", [&] {
-                k_temb_in_sigma<T><<<(d + 7) / 8, 256, 0, st>>>((const T *)w->w_t1, sigmas, step, t_per_sigma, K0, d,
-                                                               a1);
+                launch_dep(k_temb_in_sigma<T>, dim3((d + 7) / 8), dim3(256), 0, st, nullptr, (const T *)w->w_t1, sigmas,
+                           step, t_per_sigma, K0, d, a1);
             });
         L.run("gemv", [&] {
-            k_gemv2<T><<<(d + 7) / 8, 256, xs, st>>>((const T *)w->w_t2, d, e, (const T *)w->w_t2, 0, e, a1, d, 0);
+            launch_dep(k_gemv2<T>, dim3((d + 7) / 8), dim3(256), xs, st, nullptr, (const T *)w->w_t2, d, e,
+                       (const T *)w->w_t2, 0, e, (const float *)a1, d, 0);
         });
         L.run("gemv", [&] {
-            k_gemv2<T><<<(nch * d + d + 7) / 8, 256, xs, st>>>((const T *)w->w_mod, nch * d, mod_row,
-                                                               (const T *)w->w_fin, d, scale_final, e, d, 1);
+            launch_dep(k_gemv2<T>, dim3((nch * d + d + 7) / 8), dim3(256), xs, st, nullptr, (const T *)w->w_mod,
+                       nch * d, mod_row, (const T *)w->w_fin, d, scale_final, (const float *)e, d, 1);
         });
     };
     if (c->dtype == QI21_DTYPE_BF16)
@@ -916,7 +950,7 @@ extern "C" qi21_status qi21_euler_update(const float *x_k, const float *v, doubl
     cudaStream_t st = (cudaStream_t)stream;
     Launcher L(st);
     const float dsig = (float)(sigma_k1 - sigma_k);
-    L.run("euler", [&] { k_euler<<<grid_for((n + 3) / 4, 256), 256, 0, st>>>(x_k, v, dsig, x_out, n); });
+    L.run("euler", [&] { launch_dep(k_euler, dim3(grid_for((n + 3) / 4, 256)), dim3(256), 0, st, nullptr, x_k, v, dsig, x_out, n); });
     return finish(L);
 }
 
@@ -1003,7 +1037,10 @@ extern "C" qi21_status qi21_euler_update_at(const float *x_k, const float *v, co
     if (n == 0) return QI21_OK;
     cudaStream_t st = (cudaStream_t)stream;
     Launcher L(st);
-    L.run("euler", [&] { k_euler_sigma<<<grid_for((n + 3) / 4, 256), 256, 0, st>>>(x_k, v, sigmas, step, x_out, n); });
+    L.run("euler", [&] {
+        launch_dep(k_euler_sigma, dim3(grid_for((n + 3) / 4, 256)), dim3(256), 0, st, nullptr, x_k, v, sigmas, step, x_out,
+                   n);
+    });
     return finish(L);
 }
 

@@ -65,22 +65,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for part of the softmax exponentials (the MUFU unit
-// takes the rest): x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f from a
-// cubic with constant term 1 (coefficients: exp2_poly_fit.py, a least-squares
-// relative-error fit, max relative error 1.1e-4 — P is rounded to bf16
-// afterwards, relative step 2^-8); 2^n is added to the exponent field. Inputs
-// below -127 (masked keys: -inf) give exactly +0 (n = -127, f = 0, p = 1).
-__device__ __forceinline__ float ex2_poly(float x) {
-    x = fmaxf(x, -127.f);
-    const float t = x + 12582912.f;            // 1.5 * 2^23: t's low mantissa bits hold rint(x)
-    const float f = x - (t - 12582912.f);
-    float p = fmaf(0.054592825f, f, 0.24221784f);
-    p = fmaf(p, f, 0.6933686f);
-    p = fmaf(p, f, 1.0f);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 // Packed pairs of fp32 (sm_100a f32x2 arithmetic: one instruction for two lanes).
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
     uint64_t r;
@@ -113,8 +97,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // 2^x for a pair on the FMA pipe: x = n + f, n = rint(x), f in [-1/2, 1/2];
 // 2^f from a cubic with constant term 1 (least-squares relative-error fit on
-// [-1/2, 1/2], max relative error 1.1e-4; P is rounded to bf16 afterwards,
-// relative step 2^-8) and 2^n added to the exponent field. Inputs are clamped
+// [-1/2, 1/2], max relative error 1.1e-4; the coefficients are printed by
+// exp2_poly_fit.py beside this file; P is rounded to bf16 afterwards, relative
+// step 2^-8) and 2^n added to the exponent field. Inputs are clamped
 // at -127, where f = 0 and the result is exactly +0 (masked keys: -inf).
 __device__ __forceinline__ void ex2_poly2(float x0, float x1, float &e0, float &e1) {
     const uint64_t x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
@@ -171,16 +156,12 @@ struct AttnCfg {
 // Rescale the O row only when the running max grows by more than this (log2 units).
 constexpr float kRescaleLog2 = 8.0f;
 
-// Every POLY-th exponential of a row (POLY > 0) runs on the FMA pipe.
-#ifndef QI21_ATTN_EXP_POLY
-#define QI21_ATTN_EXP_POLY 0
-#endif
-#ifndef QI21_ATTN_PACKED
-#define QI21_ATTN_PACKED 0
-#endif
-#ifndef QI21_ATTN_POLY
-#define QI21_ATTN_POLY 0
-#endif
+// Every kPolyEvery-th pair of exponentials of a row runs on the FMA pipe
+// (ex2_poly2), the rest on the MUFU unit, which would otherwise take as long as
+// the MMAs per key tile. Same-GPU A/B on the single-block workload (attention
+// time over the gate/up GEMM's, interleaved runs): every 8th pair -6 %, every
+// 4th -5 %, every 2nd +6 %, against the scalar MUFU-only softmax.
+constexpr int kPolyEvery = 8;
 
 template <int DH>
 __global__ void __launch_bounds__(320, 1)
@@ -239,6 +220,8 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_launch_dependents();
+    pdl_wait();
     // keys this CTA needs: the largest limit over its query rows
     if (threadIdx.x >= 64 && threadIdx.x < 64 + C::BQ) {
         const int row = q0 + (threadIdx.x - 64);
@@ -415,7 +398,7 @@ __global__ void __launch_bounds__(320, 1)
                 for (int i = 0; i < 128; ++i)
                     if (key0 + i >= klim) sv[i >> 5][i & 31] = -INFINITY;
             }
-#if QI21_ATTN_PACKED
+            // row max: three-input max over pairs, four independent chains
             float m4[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) m4[i] = fmaxf(sv[0][2 * i], sv[0][2 * i + 1]);
@@ -423,15 +406,6 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = 8; i < 128; i += 2) m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], sv[i >> 5][i & 31],
                                                                       sv[i >> 5][(i + 1) & 31]);
             const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
-#else
-            float m8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = sv[0][i];
-#pragma unroll
-            for (int i = 8; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i >> 5][i & 31]);
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-#endif
             // move the running max only when this tile raises it by more than 2^8
             const bool first = (m_run == -INFINITY);
             const bool grow = first || (mx - m_run) * c > kRescaleLog2;
@@ -441,16 +415,11 @@ __global__ void __launch_bounds__(320, 1)
             m_run = m_new;
             // a row with no allowed key so far (half B past its limit) keeps m = -inf: P = 0
             const float mc = m_run == -INFINITY ? 0.f : m_run * c;
-#if QI21_ATTN_PACKED
+            // row sum in packed pairs (f32x2 adds), four independent chains
             uint64_t s4[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) s4[i] = 0ull;      // pairs of +0.f
             const uint64_t c2 = f2_pack(c, c), nmc2 = f2_pack(-mc, -mc);
-#else
-            float s8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) s8[i] = 0.f;
-#endif
             // P ready for the PV MMA, in two parts: keys 0..63, then 64..127
             auto signal_p = [&](int part) {
                 tmem_wait_st();
@@ -460,43 +429,19 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t u[16];
-#if QI21_ATTN_PACKED
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
-                    float x0, x1, e0, e1;
+                    float x0, x1, e0, e1;     // x = S c - m c, one f32x2 FMA for the pair (masked: -inf -> 0)
                     f2_unpack(f2_fma(f2_pack(sv[cc][2 * q], sv[cc][2 * q + 1]), c2, nmc2), x0, x1);
-#if QI21_ATTN_POLY > 0
-                    if ((cc * 16 + q) % QI21_ATTN_POLY == QI21_ATTN_POLY - 1) {
+                    if ((cc * 16 + q) % kPolyEvery == kPolyEvery - 1) {
                         ex2_poly2(x0, x1, e0, e1);
-                    } else
-#endif
-                    {
+                    } else {
                         e0 = ex2_approx(x0);
                         e1 = ex2_approx(x1);
                     }
-                    const uint64_t e2 = f2_pack(e0, e1);
-                    s4[q & 3] = f2_add(s4[q & 3], e2);
+                    s4[q & 3] = f2_add(s4[q & 3], f2_pack(e0, e1));
                     u[q] = pack_bf16x2(e0, e1);
                 }
-#else
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    float e[2];
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const float x = fmaf(sv[cc][2 * q + t], c, -mc);   // masked: -inf -> 0
-#if QI21_ATTN_EXP_POLY > 0
-                        e[t] = ((2 * q + t) % QI21_ATTN_EXP_POLY == QI21_ATTN_EXP_POLY - 1) ? ex2_poly(x)
-                                                                                          : ex2_approx(x);
-#else
-                        e[t] = ex2_approx(x);
-#endif
-                    }
-                    s8[(2 * q) & 7] += e[0];
-                    s8[(2 * q + 1) & 7] += e[1];
-                    u[q] = pack_bf16x2(e[0], e[1]);
-                }
-#endif
                 tmem_st16(t_s + cc * 16, u);               // P_h: keys 32cc .. 32cc+31
                 if (cc == 1) {
                     // O rescale (rare) before the first P signal, so that PV_h(j) sees the
@@ -518,14 +463,10 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
             signal_p(1);
-#if QI21_ATTN_PACKED
             const uint64_t s2 = f2_add(f2_add(s4[0], s4[1]), f2_add(s4[2], s4[3]));
             float sa, sb;
             f2_unpack(s2, sa, sb);
             l_run += sa + sb;
-#else
-            l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-#endif
         }
         // merge the halves: each publishes its (m, l) per row; half h then writes
         // output columns [h Dh/2, (h+1) Dh/2) of its rows from O_A and O_B

@@ -43,6 +43,16 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialisation attribute may be scheduled while the kernel before it in
+// the stream is still running; pdl_wait() returns once every preceding kernel
+// has completed and its memory is visible, so a kernel calls it before its
+// first global-memory access (after any prologue that touches only its own
+// shared memory, TMEM and kernel parameters). pdl_launch_dependents() allows
+// the next kernel to be scheduled. Both are no-ops in a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Error word in the workspace: kernels set a code and return instead of
 // trapping; the host reads it with qi21_check_device_error.
 enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_LAYOUT = 2 };

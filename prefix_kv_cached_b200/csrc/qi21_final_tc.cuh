@@ -44,6 +44,8 @@ struct FinalParams {
 // (16-byte loads and stores), d % 8 == 0.
 static __global__ void __launch_bounds__(256) k_final_prep(const bf16 *__restrict__ w_out, const float *__restrict__ sf,
                                                            int d, bf16 *__restrict__ wp, float *__restrict__ u) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ float red[32];
     const int c = blockIdx.x;
     const uint4 *w8 = reinterpret_cast<const uint4 *>(w_out + (size_t)c * d);
@@ -117,6 +119,8 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -230,6 +234,8 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
 static __global__ void __launch_bounds__(256) k_final_reduce(const float *__restrict__ part, int ksplit, int R, int d,
                                                              const float *__restrict__ u, float eps,
                                                              float *__restrict__ v) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int row = t >> 4, g = t & 15;
     if (row >= R) return;

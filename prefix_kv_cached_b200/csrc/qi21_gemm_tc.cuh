@@ -245,6 +245,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if constexpr (PAIR) cluster_sync();   // the peer's barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer

@@ -15,6 +15,8 @@ namespace qi21 {
 // ---------------------------------------------------------------------------
 static __global__ void k_prep_gates(const float *__restrict__ mod_lo, const float *__restrict__ mod_hi, int d,
                              int use_shift, float *__restrict__ gates) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int g1 = use_shift ? 2 : 1, g2 = use_shift ? 5 : 3;
     for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < d; c += gridDim.x * blockDim.x) {
         gates[0 * d + c] = tanhf(mod_lo[g1 * d + c]);
@@ -36,6 +38,8 @@ __global__ void __launch_bounds__(256) k_modln_vec(const float *__restrict__ h, 
                                                    const float *__restrict__ scale_hi,
                                                    const float *__restrict__ shift_lo,
                                                    const float *__restrict__ shift_hi, float eps) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ float red[32];
     const int r = blockIdx.x;
     const int m = r % M;
@@ -635,6 +639,8 @@ __device__ __forceinline__ void euler_body(const float *__restrict__ x, const fl
 
 static __global__ void k_euler(const float *__restrict__ x, const float *__restrict__ v, float dsig,
                         float *__restrict__ xo, int64_t n) {
+    pdl_launch_dependents();
+    pdl_wait();
     euler_body(x, v, dsig, xo, n);
 }
 
@@ -642,6 +648,8 @@ static __global__ void k_euler(const float *__restrict__ x, const float *__restr
 // difference is formed in fp64 and rounded once, as on the host path.
 static __global__ void k_euler_sigma(const float *__restrict__ x, const float *__restrict__ v,
                                      const double *__restrict__ sigmas, int step, float *__restrict__ xo, int64_t n) {
+    pdl_launch_dependents();
+    pdl_wait();
     euler_body(x, v, (float)(sigmas[step + 1] - sigmas[step]), xo, n);
 }
 
@@ -693,6 +701,8 @@ __device__ __forceinline__ float dot_row(const T *__restrict__ w, const float *_
 template <typename T>
 __global__ void __launch_bounds__(256) k_temb_in(const T *__restrict__ W, TembArg emb, int K, int N,
                                                  float *__restrict__ y) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ float xs[512];
     for (int k = threadIdx.x; k < K; k += blockDim.x) xs[k] = emb.v[k];
     __syncthreads();
@@ -712,6 +722,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_temb_in_sigma(const T *__restrict__ W, const double *__restrict__ sigmas,
                                                        int step, double t_per_sigma, int K, int N,
                                                        float *__restrict__ y) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ float xs[512];
     const int half = K / 2;
     const double t = t_per_sigma * sigmas[step];
@@ -734,6 +746,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_gemv2(const T *__restrict__ W1, int N1, float *__restrict__ y1,
                                                const T *__restrict__ W2, int N2, float *__restrict__ y2,
                                                const float *__restrict__ x, int K, int silu_in) {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ float xs[];
     for (int k = threadIdx.x; k < K; k += blockDim.x) xs[k] = silu_in ? silu_f(x[k]) : x[k];
     __syncthreads();

@@ -94,7 +94,10 @@ def test_packed_prefix_feeds_the_extract(B, mode):
 @pytest.mark.parametrize("dtype_name", ["float32", "bfloat16"])
 def test_pack_weights_from_canonical_layout(B, dtype_name):
     """qi21_pack_weights: canonical [in][out] weights become exactly the [out][in]
-    tensors the kernels read, and a cached step through them is bit-identical."""
+    tensors the kernels read (bit-exact), and a cached step through them gives
+    the same result (to the run-to-run variation of the residual GEMMs, whose
+    partial sums reach h in a non-deterministic order: rel-L2 < 1e-3; a
+    packing mistake moves it by order 1)."""
     from prefix_kv_cached_b200.runner import Qi21Runner
     w = C.make_workload("small")
     dtype = B.QI21_DTYPE_F32 if dtype_name == "float32" else B.QI21_DTYPE_BF16
@@ -132,4 +135,5 @@ def test_pack_weights_from_canonical_layout(B, dtype_name):
         torch.cuda.synchronize()
         outs.append(v.clone())
     r.check_device()
-    assert torch.equal(outs[0], outs[1])
+    a, b = outs[0].double(), outs[1].double()
+    assert float(torch.linalg.norm(a - b) / torch.linalg.norm(b)) < 1e-3
