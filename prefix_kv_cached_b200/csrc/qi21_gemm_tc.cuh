@@ -30,7 +30,17 @@ constexpr int TC_THREADS = 192;
 // shared memory (two buffers per warp) for the TMA reduce-add into the
 // residual stream, or the TMA store.
 constexpr int TC_RED_BUF = 32 * 32 * 4;
-constexpr int TC_RED_BYTES = 4 * 2 * TC_RED_BUF;
+// staging boxes per epilogue warp: 2 for the residual (its GEMMs are bound by the
+// MMAs), 6 for the store epilogue (img_in, K = 64: bound by the stores; each box
+// waits for the TMA engine to read it before it is written again)
+template <int EPI>
+__host__ __device__ constexpr int tc_red_nbuf() {
+    return EPI == EPI_STORE ? 6 : 2;
+}
+template <int EPI>
+__host__ __device__ constexpr int tc_red_bytes() {
+    return 4 * tc_red_nbuf<EPI>() * TC_RED_BUF;
+}
 template <int EPI>
 __host__ __device__ constexpr bool tc_boxed_epilogue() {
     return EPI == EPI_RESIDUAL || EPI == EPI_STORE;
@@ -46,10 +56,10 @@ struct TcCfg {
     static constexpr int B_ROWS = PAIR ? 128 : 256;                 // W rows a CTA loads per K block
     static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
     static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
-    static constexpr int STAGES = PAIR ? (tc_boxed_epilogue<EPI>() ? 5 : 6) : 4;
+    static constexpr int STAGES = EPI == EPI_STORE ? 2 : (PAIR ? (tc_boxed_epilogue<EPI>() ? 5 : 6) : 4);
     static constexpr int TILE_ROWS = PAIR ? 256 : 128;              // output rows of a work unit
     static constexpr size_t SMEM =
-        1024 + (size_t)STAGES * STAGE_BYTES + (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0) + 256;
+        1024 + (size_t)STAGES * STAGE_BYTES + (tc_boxed_epilogue<EPI>() ? tc_red_bytes<EPI>() : 0) + 256;
 };
 template <int EPI, bool PAIR>
 constexpr size_t tc_smem_bytes() {
@@ -105,7 +115,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src,
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_group_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -198,7 +212,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *stage_base = smem;
     uint8_t *red_base = smem + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(red_base + (tc_boxed_epilogue<EPI>() ? TC_RED_BYTES : 0));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(red_base + (tc_boxed_epilogue<EPI>() ? tc_red_bytes<EPI>() : 0));
     uint64_t *full = bars, *empty = bars + Cfg::STAGES, *tfull = bars + 2 * Cfg::STAGES, *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -405,7 +419,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 // and one lane reduce-adds (or stores) the box.
                 const int n0 = n_blk * TC_BN;
                 const float *g = EPI == EPI_RESIDUAL ? (m < p.split ? p.g_lo : p.g_hi) + n0 : nullptr;
-                uint8_t *stg = red_base + (size_t)(warp - 2) * 2 * TC_RED_BUF;
+                constexpr int NBUF = tc_red_nbuf<EPI>();
+                uint8_t *stg = red_base + (size_t)(warp - 2) * NBUF * TC_RED_BUF;
                 const int sw = lane & 7;
                 const int box_row = m_blk * Cfg::TILE_ROWS + (int)rank * TC_BM + quad * 32;
 #pragma unroll 1
@@ -424,9 +439,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             v[4 * i + 3] *= gv.w;
                         }
                     }
-                    uint8_t *buf = stg + (red_count & 1) * TC_RED_BUF;
-                    if (red_count >= 2) {
-                        if (lane == 0) bulk_wait_group_read1();   // the reduce that used `buf` has read it
+                    uint8_t *buf = stg + (red_count % NBUF) * TC_RED_BUF;
+                    if (red_count >= NBUF) {
+                        if (lane == 0) bulk_wait_group_read<NBUF - 1>();   // the copy that used `buf` has read it
                         __syncwarp();
                     }
                     uint8_t *rowp = buf + lane * 128;
